@@ -1,0 +1,205 @@
+"""Seeded synthetic inputs for the attention forward workloads.
+
+This module only draws random numbers and lays them out; it holds none of
+the attention arithmetic. Both the fp64 oracle (under ``oracle/``) and the
+CUDA path consume what it returns, so it is the one module they share.
+
+Recipe (every value i.i.d. N(0, 1) unless stated):
+  * a ``torch.Generator('cpu')`` seeded with the workload's seed;
+  * ``torch.randn(shape, dtype=float32, generator=g)`` drawn in the order
+    q, k, v (MLA decode: q, kv);
+  * then a cast to the workload's dtype with round-to-nearest-even.
+The shapes follow the pages' own workloads: the flash_attn layouts
+``[B, S, H, D]`` / ``[total_tokens, H, D]`` of mxflashattn 1.4.0
+(``flash_attn_func``, ``flash_attn_varlen_func``) and the MLA decode inputs
+``(q, kv, qo_indptr, kv_indptr)`` of kernelbot-amd-mixed-mla submission
+588924 (``custom_kernel``).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+
+
+@dataclass
+class Problem:
+    """One attention forward problem in packed (varlen) form.
+
+    q: [total_q, Hq, Dqk]; k: [total_k, Hkv, Dqk]; v: [total_k, Hkv, Dv]
+    (for MLA decode k and v are views of one kv tensor [total_k, 1, 576]).
+    cu_q / cu_k: int32 [batch + 1] cumulative lengths.
+    ``batched`` is set when every sequence has the same length, so the
+    tensors can also be viewed as [B, S, H, D].
+    """
+
+    name: str
+    dtype: str
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    cu_q: torch.Tensor
+    cu_k: torch.Tensor
+    hq: int
+    hkv: int
+    dqk: int
+    dv: int
+    causal: bool
+    scale: float
+    batched: bool = False
+    mla: bool = False
+    kv: torch.Tensor | None = None  # MLA: the single [total_k, 576] cache
+    check_rows: torch.Tensor | None = None  # [n, 2] (token, head) pairs the oracle evaluates
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def batch(self) -> int:
+        return self.cu_q.numel() - 1
+
+    @property
+    def total_q(self) -> int:
+        return int(self.cu_q[-1])
+
+    @property
+    def total_k(self) -> int:
+        return int(self.cu_k[-1])
+
+    def seqlens_q(self) -> list[int]:
+        c = self.cu_q.tolist()
+        return [c[i + 1] - c[i] for i in range(len(c) - 1)]
+
+    def seqlens_k(self) -> list[int]:
+        c = self.cu_k.tolist()
+        return [c[i + 1] - c[i] for i in range(len(c) - 1)]
+
+
+def _cu(lengths: list[int]) -> torch.Tensor:
+    out = [0]
+    for n in lengths:
+        out.append(out[-1] + int(n))
+    return torch.tensor(out, dtype=torch.int32)
+
+
+def _randn(g: torch.Generator, shape, dtype: str) -> torch.Tensor:
+    return torch.randn(shape, dtype=torch.float32, generator=g).to(DTYPES[dtype])
+
+
+def batched(seed: int, B: int, Sq: int, Sk: int, Hq: int, Hkv: int, D: int, dtype: str,
+            causal: bool, scale: float | None = None, name: str = "batched",
+            Dv: int | None = None) -> Problem:
+    """[B, S, H, D] inputs, stored packed as [B*S, H, D]."""
+    Dv = D if Dv is None else Dv
+    g = torch.Generator("cpu").manual_seed(seed)
+    q = _randn(g, (B, Sq, Hq, D), dtype).reshape(B * Sq, Hq, D)
+    k = _randn(g, (B, Sk, Hkv, D), dtype).reshape(B * Sk, Hkv, D)
+    v = _randn(g, (B, Sk, Hkv, Dv), dtype).reshape(B * Sk, Hkv, Dv)
+    return Problem(name, dtype, q, k, v, _cu([Sq] * B), _cu([Sk] * B), Hq, Hkv, D, Dv, causal,
+                   D ** -0.5 if scale is None else scale, batched=True,
+                   meta={"B": B, "Sq": Sq, "Sk": Sk})
+
+
+def varlen(seed: int, lens_q: list[int], lens_k: list[int], Hq: int, Hkv: int, D: int, dtype: str,
+           causal: bool, scale: float | None = None, name: str = "varlen") -> Problem:
+    g = torch.Generator("cpu").manual_seed(seed)
+    tq, tk = sum(lens_q), sum(lens_k)
+    q = _randn(g, (tq, Hq, D), dtype)
+    k = _randn(g, (tk, Hkv, D), dtype)
+    v = _randn(g, (tk, Hkv, D), dtype)
+    return Problem(name, dtype, q, k, v, _cu(lens_q), _cu(lens_k), Hq, Hkv, D, D, causal,
+                   D ** -0.5 if scale is None else scale)
+
+
+def mla_decode(seed: int, batch: int, q_len: int, kv_len: int, heads: int = 16, dqk: int = 576,
+               dv: int = 512, dtype: str = "bf16", name: str = "mla_decode",
+               lens_kv: list[int] | None = None) -> Problem:
+    """MLA decode: q [batch*q_len, heads, 576]; one shared kv head [total_kv, 576];
+    k = kv[:, :576], v = kv[:, :512] (kernelbot-amd-mixed-mla 588924, ``_flash_fused``)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    lens_kv = [kv_len] * batch if lens_kv is None else lens_kv
+    tk = sum(lens_kv)
+    q = _randn(g, (batch * q_len, heads, dqk), dtype)
+    kv = _randn(g, (tk, dqk), dtype)
+    k = kv.view(tk, 1, dqk)
+    v = kv[:, :dv].view(tk, 1, dv)  # a strided view: row stride 576
+    return Problem(name, dtype, q, k, v, _cu([q_len] * batch), _cu(lens_kv), heads, 1, dqk, dv,
+                   False, dqk ** -0.5, mla=True, kv=kv,
+                   meta={"batch": batch, "q_len": q_len, "kv_len": kv_len})
+
+
+# ---------------------------------------------------------------------------
+# The five named workloads.
+# ---------------------------------------------------------------------------
+
+def cfg_single_head_fp32() -> Problem:
+    """fp32, B=1, H=1, Sq=Sk=128, D=64, non-causal, scale 1/8; seed 0."""
+    return batched(0, 1, 128, 128, 1, 1, 64, "f32", False, 1.0 / math.sqrt(64),
+                   name="single_head_fp32_b1_h1_s128_d64")
+
+
+def cfg_batched_causal(B: int = 4, S: int = 2048, H: int = 16, D: int = 128, dtype: str = "bf16") -> Problem:
+    """bf16, B=4, Hq=Hkv=16, Sq=Sk=2048, D=128, causal, default scale; seed 1."""
+    return batched(1, B, S, S, H, H, D, dtype, True, None,
+                   name=f"batched_causal_b{B}_h{H}_s{S}_d{D}_{dtype}")
+
+
+def varlen_lengths(seed: int = 2, n: int = 16, lo: int = 128, hi: int = 4096) -> tuple[torch.Generator, list[int]]:
+    g = torch.Generator("cpu").manual_seed(seed)
+    lens = torch.randint(lo, hi + 1, (n,), generator=g).tolist()
+    return g, lens
+
+
+def cfg_varlen_gqa() -> Problem:
+    """bf16 varlen GQA causal: 16 sequences, lengths U[128, 4096] (seed 2),
+    cu_seqlens_q = cu_seqlens_k, Hq=32, Hkv=8, D=128; q,k,v drawn from the
+    same generator right after the lengths."""
+    g, lens = varlen_lengths()
+    t = sum(lens)
+    q = _randn(g, (t, 32, 128), "bf16")
+    k = _randn(g, (t, 8, 128), "bf16")
+    v = _randn(g, (t, 8, 128), "bf16")
+    cu = _cu(lens)
+    return Problem("varlen_gqa_causal_16seq_hq32_hkv8_d128_bf16", "bf16", q, k, v, cu, cu.clone(),
+                   32, 8, 128, 128, True, 128 ** -0.5, meta={"lens": lens})
+
+
+def cfg_mla_decode() -> Problem:
+    """MLA split-KV decode, bf16: batch 128, q_len 4, 16 heads, 576/512, kv_len 8192; seed 3."""
+    return mla_decode(3, 128, 4, 8192, name="mla_decode_b128_q4_h16_kv8192_bf16")
+
+
+def cfg_long_causal(S: int = 32768, H: int = 32, rows_per_head: int = 256) -> Problem:
+    """bf16, B=1, Hq=Hkv=32, Sq=Sk=32768, D=128, causal; seed 4. After q,k,v the
+    same generator draws randperm(S)[:256] per head; rows 0 and S-1 are added."""
+    g = torch.Generator("cpu").manual_seed(4)
+    q = _randn(g, (S, H, 128), "bf16")
+    k = _randn(g, (S, H, 128), "bf16")
+    v = _randn(g, (S, H, 128), "bf16")
+    pairs = []
+    for h in range(H):
+        rows = torch.randperm(S, generator=g)[:rows_per_head].tolist()
+        for r in sorted(set(rows) | {0, S - 1}):
+            pairs.append((r, h))
+    cu = _cu([S])
+    return Problem(f"long_causal_b1_h{H}_s{S}_d128_bf16", "bf16", q, k, v, cu, cu.clone(), H, H, 128, 128,
+                   True, 128 ** -0.5, batched=True, check_rows=torch.tensor(pairs, dtype=torch.int64),
+                   meta={"B": 1, "Sq": S, "Sk": S})
+
+
+def sample_rows(p: Problem, n_per_head: int, seed: int) -> torch.Tensor:
+    """(token, head) pairs for a sampled oracle check: n random tokens per head,
+    plus the first and last token of every sequence."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    ends = set()
+    c = p.cu_q.tolist()
+    for b in range(p.batch):
+        if c[b + 1] > c[b]:
+            ends |= {c[b], c[b + 1] - 1}
+    pairs = []
+    for h in range(p.hq):
+        rows = torch.randint(0, p.total_q, (n_per_head,), generator=g).tolist()
+        for r in sorted(set(rows) | ends):
+            pairs.append((r, h))
+    return torch.tensor(pairs, dtype=torch.int64)
