@@ -1,0 +1,166 @@
+/*
+ * mxfa.h -- C ABI of the fused attention forward library (libmxfa.so).
+ *
+ * Every entry point computes, per query row i of sequence b and query head h,
+ *
+ *     O[i,h,:] = sum_j P_ij * v[j, h/G, :],   P_ij = exp(s_ij - m_i) / l_i
+ *     s_ij     = softmax_scale * <q[i,h,:], k[j, h/G, :]>   for j visible,
+ *     LSE[i,h] = m_i + ln(l_i)                 (natural log, fp32)
+ *
+ * without materialising the score matrix: KV is consumed tile by tile with a
+ * running max, running sum and rescaled accumulator (the online softmax of
+ * mxflashattn 1.4.0 prefill.py, prefill_chunked_reference, and of
+ * oxillama-runtime 0.1.0 flash_attention.rs, flash_attention).
+ *
+ *   - G = Hq / Hkv: q head h reads kv head h / G (grouped-query attention,
+ *     oxillama-runtime flash_attention.rs, flash_attention_gqa).
+ *   - causal: key j is visible to query i of a sequence with Sq queries and
+ *     Sk keys iff j <= i + Sk - Sq (bottom-right alignment, mxflashattn
+ *     prefill.py); keys j >= Sk are never visible.
+ *   - A row with no visible key gets O = 0 and LSE = -inf.
+ *   - softmax_scale: pass NaN for the default Dqk^-0.5 (mxflashattn api.py,
+ *     _resolved_scale); 0.0 is a legal scale (uniform attention).
+ *
+ * Conventions shared by all entry points
+ *   Pointers: q, k, v, o, lse, cu_seqlens / indptr arrays and workspace are
+ *     DEVICE pointers owned by the caller; the library never allocates,
+ *     frees or synchronises.  q, k, v, o must be 16-byte aligned and every
+ *     row/head stride must be a multiple of 16 bytes.  lse may be NULL (not
+ *     written).
+ *   Dtypes: q, k, v and o share one dtype (mxfa_dtype_t); lse is fp32.
+ *   Stream: the work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Nothing is launched when a check fails.
+ *   Errors: the return value is MXFA_OK or an error code; mxfa_last_error()
+ *     returns a message for the calling thread's last failure.  Faults that
+ *     can only be seen on the device (a bounded wait that ran out) are
+ *     recorded in the workspace status word, read by
+ *     mxfa_read_device_status().
+ *   Workspace: each call needs `workspace` of at least the size returned by
+ *     the matching *_workspace_size function (256-byte aligned device
+ *     memory).  It holds the status word, the tile schedule and, for decode,
+ *     the split partials.  Calls that share one workspace must be ordered on
+ *     the device (same stream, or synchronised).
+ *   Strict mode: with the environment variable MXFA_STRICT_VALIDATION=1 the
+ *     varlen and decode entry points copy cu_seqlens / indptr to the host
+ *     and check them (start at 0, non-decreasing, end at the totals, lengths
+ *     within the stated maxima), as mxflashattn api.py does under
+ *     MXFLASHATTN_STRICT_VALIDATION.  This synchronises the stream.
+ */
+#ifndef MXFA_H
+#define MXFA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MXFA_OK = 0,
+  MXFA_ERR_INVALID_ARG = 1,  /* bad pointer, size, stride or alignment */
+  MXFA_ERR_UNSUPPORTED = 2,  /* legal but not implemented (head dim, dtype) */
+  MXFA_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small */
+  MXFA_ERR_CUDA = 4,         /* a CUDA runtime call failed */
+  MXFA_ERR_TIMEOUT = 5       /* a device-side bounded wait ran out */
+} mxfa_status_t;
+
+typedef enum { MXFA_F32 = 0, MXFA_F16 = 1, MXFA_BF16 = 2 } mxfa_dtype_t;
+
+/*
+ * Batched attention forward, layout [B, S, H, D]
+ * (mxflashattn 1.4.0 api.py, flash_attn_func).
+ *   q: [B, Sq, Hq, D]   element (b,i,h,d) at b*Sq*q_row_stride + i*q_row_stride + h*q_head_stride + d
+ *   k: [B, Sk, Hkv, D]  likewise with k_row_stride / k_head_stride (v the same with v_*)
+ *   o: [B, Sq, Hq, D]   written; o_row_stride / o_head_stride
+ *   lse: [B, Sq, Hq] fp32, contiguous (or NULL)
+ * Strides are in elements; the batch stride is S * row stride (batches are
+ * contiguous); the last dimension is contiguous.
+ * Supported: D in {64, 128}; dtypes bf16 and f16 run on the tensor-core
+ * kernel, f32 on the exact CUDA-core kernel; Hq a positive multiple of Hkv.
+ * Sq = 0 or B = 0 is a no-op; Sk = 0 gives O = 0, LSE = -inf.
+ */
+size_t mxfa_attn_fwd_workspace_size(int B, int Sq, int Sk, int Hq, int Hkv, int D, mxfa_dtype_t dtype);
+mxfa_status_t mxfa_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                            int B, int Sq, int Sk, int Hq, int Hkv, int D, mxfa_dtype_t dtype,
+                            int64_t q_row_stride, int64_t q_head_stride,
+                            int64_t k_row_stride, int64_t k_head_stride,
+                            int64_t v_row_stride, int64_t v_head_stride,
+                            int64_t o_row_stride, int64_t o_head_stride,
+                            float softmax_scale, int causal,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Variable-length attention forward, packed layout [total_tokens, H, D]
+ * (mxflashattn 1.4.0 api.py, flash_attn_varlen_func; lattice-inference
+ * 0.7.1 standard.rs, multi_head_attention_batched: cu_seqlens has batch+1
+ * entries, starts at 0 and ends at the total).
+ *   q: [total_q, Hq, D], k/v: [total_k, Hkv, D], o: [total_q, Hq, D] -- contiguous
+ *   lse: [total_q, Hq] fp32 (or NULL)
+ *   cu_seqlens_q / cu_seqlens_k: DEVICE int32 arrays of batch+1 entries;
+ *   sequence b holds tokens [cu[b], cu[b+1]).  max_seqlen_q / max_seqlen_k
+ *   must bound every sequence length (they size the schedule; values beyond
+ *   them are an error caught in strict mode and otherwise undefined).
+ * Supported as mxfa_attn_fwd.  Empty query sequences are skipped; a
+ * sequence with no keys gives O = 0 and LSE = -inf.
+ */
+size_t mxfa_attn_varlen_fwd_workspace_size(int batch, int max_seqlen_q, int max_seqlen_k, int Hq, int D,
+                                           mxfa_dtype_t dtype);
+mxfa_status_t mxfa_attn_varlen_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                   int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                                   int Hq, int Hkv, int D, mxfa_dtype_t dtype,
+                                   float softmax_scale, int causal,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Split-KV decode (few queries per sequence, long KV), with the partial
+ * (accumulator, max, sum) combine of kernelbot-amd-mixed-mla submission
+ * 588924 (_flash_splitk / _reduce_splitk).
+ *   q: [total_q, Hq, Dqk] contiguous; sequence b owns queries
+ *      [qo_indptr[b], qo_indptr[b+1]) and keys [kv_indptr[b], kv_indptr[b+1])
+ *   k: key row t, head g at k + t*k_row_stride + g*Dqk  (Dqk contiguous)
+ *   v: value row t, head g at v + t*v_row_stride + g*Dv (Dv contiguous)
+ *   o: [total_q, Hq, Dv] contiguous; lse: [total_q, Hq] fp32 (or NULL)
+ *   qo_indptr / kv_indptr: DEVICE int32, batch+1 entries each.
+ * MLA (DeepSeek-style latent cache): k = v = the kv base pointer, Hkv = 1,
+ * Dqk = 576, Dv = 512, k_row_stride = v_row_stride = 576: value = first 512
+ * columns of each cached row; the tensor-core kernel reads each KV tile once
+ * and uses it as both operands.  That path needs bf16/f16 and
+ * max_q_len * Hq <= 64.  Other shapes ((Dqk, Dv) = (64, 64) or (128, 128),
+ * or f32) run on the exact CUDA-core kernel.
+ * num_splits: 0 = automatic (the KV of all sequences is cut into
+ *   near-equal pieces, one run per SM); k >= 1 = every sequence's KV is cut
+ *   into k pieces.  The result does not depend on it beyond fp32 rounding.
+ */
+size_t mxfa_attn_decode_splitkv_workspace_size(int batch, int max_q_len, int Hq, int Dv, int max_kv_len,
+                                               int num_splits, mxfa_dtype_t dtype);
+mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                                       const int32_t *qo_indptr, const int32_t *kv_indptr,
+                                       int batch, int total_q, int total_kv, int max_q_len, int max_kv_len,
+                                       int Hq, int Hkv, int Dqk, int Dv,
+                                       int64_t k_row_stride, int64_t v_row_stride,
+                                       mxfa_dtype_t dtype, float softmax_scale, int causal, int num_splits,
+                                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* Message for the calling thread's most recent failure ("" if none). */
+const char *mxfa_last_error(void);
+
+/*
+ * Synchronises `stream`, reads the status word the last call wrote into
+ * `workspace` and returns it (MXFA_OK, or MXFA_ERR_TIMEOUT when a bounded
+ * device wait gave up; the kernel then skipped its remaining work and left
+ * the outputs incomplete).  mxfa_device_status_detail() returns the site
+ * code of that wait from the same read.
+ */
+mxfa_status_t mxfa_read_device_status(const void *workspace, void *stream);
+uint32_t mxfa_device_status_detail(void);
+
+/* Library version, (major << 16) | (minor << 8) | patch. */
+uint32_t mxfa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXFA_H */

@@ -1,0 +1,114 @@
+"""The C-ABI library: it loads without a GPU, exports every function the
+header declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxfa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_attention_21_b200 import build_ext
+    import tiled_attention_21_b200 as m
+    try:
+        build_ext.build()
+    except RuntimeError as e:  # no nvcc
+        if not os.path.exists(m.LIB_PATH):
+            pytest.skip(str(e))
+    return m.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mxfa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_entry_points():
+    names = declared_functions()
+    for n in ("mxfa_attn_fwd", "mxfa_attn_varlen_fwd", "mxfa_attn_decode_splitkv", "mxfa_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from tiled_attention_21_b200 import LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(\S+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        getattr(lib, n)
+
+
+FAKE = 0x100000  # never dereferenced: every call below fails validation first
+
+
+def fwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Sq=8, Sk=8, Hq=2, Hkv=1, D=64, dt=2,
+             qr=128, qh=64, kr=64, kh=64, vr=64, vh=64, orr=128, oh=64, scale=float("nan"), causal=0,
+             ws=FAKE, wsn=4096)
+    a.update(kw)
+    return lib.mxfa_attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Sq"], a["Sk"], a["Hq"], a["Hkv"],
+                             a["D"], a["dt"], a["qr"], a["qh"], a["kr"], a["kh"], a["vr"], a["vh"], a["orr"], a["oh"],
+                             a["scale"], a["causal"], a["ws"], a["wsn"], None)
+
+
+def test_validation_errors(lib):
+    import tiled_attention_21_b200 as m
+    assert fwd(lib, Hq=3, Hkv=2) == m.MXFA_ERR_INVALID_ARG
+    assert b"multiple" in lib.mxfa_last_error()
+    assert fwd(lib, D=96) == m.MXFA_ERR_UNSUPPORTED
+    assert fwd(lib, dt=7) == m.MXFA_ERR_INVALID_ARG
+    assert fwd(lib, q=None) == m.MXFA_ERR_INVALID_ARG
+    assert fwd(lib, q=FAKE + 8) == m.MXFA_ERR_INVALID_ARG
+    assert fwd(lib, qr=100) == m.MXFA_ERR_INVALID_ARG  # 200 bytes: not a multiple of 16
+    assert fwd(lib, ws=None) == m.MXFA_ERR_WORKSPACE
+    assert fwd(lib, ws=FAKE + 16) == m.MXFA_ERR_WORKSPACE
+    assert fwd(lib, wsn=16) == m.MXFA_ERR_WORKSPACE
+    assert fwd(lib, B=-1) == m.MXFA_ERR_INVALID_ARG
+    assert fwd(lib, scale=float("inf")) == m.MXFA_ERR_INVALID_ARG
+    # empty problems are a no-op and succeed without touching the device
+    assert fwd(lib, B=0) == m.MXFA_OK
+    assert fwd(lib, Sq=0) == m.MXFA_OK
+
+
+def test_varlen_and_decode_validation(lib):
+    import tiled_attention_21_b200 as m
+    r = lib.mxfa_attn_varlen_fwd(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, 2, 10, 10, 8, 8, 4, 2, 128, 2,
+                                 float("nan"), 1, FAKE, 1 << 20, None)
+    assert r == m.MXFA_ERR_INVALID_ARG  # cu_seqlens_q NULL
+    r = lib.mxfa_attn_varlen_fwd(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 10, 10, 11, 8, 4, 2, 128, 2,
+                                 float("nan"), 1, FAKE, 1 << 20, None)
+    assert r == m.MXFA_ERR_INVALID_ARG  # max_seqlen_q > total_q
+    r = lib.mxfa_attn_decode_splitkv(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 8, 64, 4, 32, 16, 1, 576, 256,
+                                     576, 576, 2, float("nan"), 0, 0, FAKE, 1 << 20, None)
+    assert r == m.MXFA_ERR_UNSUPPORTED  # (576, 256)
+    r = lib.mxfa_attn_decode_splitkv(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 8, 64, 4, 32, 16, 1, 576, 512,
+                                     500, 576, 2, float("nan"), 0, 0, FAKE, 1 << 20, None)
+    assert r == m.MXFA_ERR_INVALID_ARG  # k row stride shorter than a row
+    r = lib.mxfa_attn_decode_splitkv(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 8, 64, 4, 32, 16, 1, 576, 512,
+                                     576, 576, 2, float("nan"), 0, -1, FAKE, 1 << 20, None)
+    assert r == m.MXFA_ERR_INVALID_ARG  # negative split count
+
+
+def test_workspace_sizes(lib):
+    assert lib.mxfa_attn_fwd_workspace_size(4, 2048, 2048, 16, 16, 128, 2) >= 256
+    small = lib.mxfa_attn_varlen_fwd_workspace_size(2, 128, 128, 8, 128, 2)
+    big = lib.mxfa_attn_varlen_fwd_workspace_size(64, 32768, 32768, 8, 128, 2)
+    assert 256 < small < big
+    assert lib.mxfa_attn_varlen_fwd_workspace_size(2, 128, 128, 8, 128, 0) == 256  # fp32 path needs no schedule
+
+
+def test_product_path_does_not_touch_the_oracle():
+    """The package never imports, loads or builds anything under oracle/."""
+    pkg = os.path.join(ROOT, "tiled_attention_21_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower(), f

@@ -1,0 +1,70 @@
+"""Parity of the split-KV decode entry point with the fp64 oracle."""
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import compare
+from runners import run, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    import tiled_attention_21_b200 as mx
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    mx.load()
+
+
+def check(p, num_splits=0, pairs=None):
+    d = to_dev(p)
+    o, l = run(p, d, num_splits=num_splits)
+    torch.cuda.synchronize()
+    if pairs is None:
+        ro, rl = oracle.problem(p)
+        return compare(o, l, ro, rl, p.q.dtype, p.name), (o, l)
+    ro, rl = oracle.problem(p, pairs=pairs)
+    return compare(o.cpu()[pairs[:, 0], pairs[:, 1]], l.cpu()[pairs[:, 0], pairs[:, 1]], ro, rl, p.q.dtype,
+                   p.name), (o, l)
+
+
+@pytest.mark.parametrize("splits", [0, 1, 2, 3, 8])
+def test_mla_small(splits):
+    p = workloads.mla_decode(21, batch=3, q_len=4, kv_len=700)
+    check(p, splits)
+
+
+def test_mla_ragged_lengths():
+    p = workloads.mla_decode(22, batch=5, q_len=4, kv_len=0, lens_kv=[1, 64, 65, 1000, 129])
+    check(p)
+
+
+def test_mla_fp16_and_small_q():
+    p = workloads.mla_decode(23, batch=4, q_len=1, kv_len=333, dtype="f16")
+    check(p)
+
+
+def test_mla_split_invariance():
+    p = workloads.mla_decode(24, batch=2, q_len=4, kv_len=2048)
+    _, (o1, l1) = check(p, 1)
+    _, (o8, l8) = check(p, 8)
+    assert (o1.float() - o8.float()).abs().max() <= 4e-3
+    assert (l1 - l8).abs().max() <= 1e-4
+
+
+@pytest.mark.parametrize("dims,dt", [((128, 128), "bf16"), ((64, 64), "f16"), ((128, 128), "f32")])
+def test_gqa_decode(dims, dt):
+    dqk, dv = dims
+    p = workloads.varlen(25, [1, 1, 2, 1], [300, 1, 77, 1024], 8, 2, dqk, dt, False)
+    d = to_dev(p)
+    o, l = run(p, d, "decode")
+    ro, rl = oracle.problem(p)
+    compare(o, l, ro, rl, p.q.dtype, "gqa decode")
+
+
+def test_full_size_mla_sampled():
+    p = workloads.cfg_mla_decode()
+    pairs = workloads.sample_rows(p, 16, 104)
+    check(p, 0, pairs)

@@ -1,0 +1,446 @@
+// mxfa.cu -- host side of the C ABI declared in include/mxfa.h.
+//
+// Validates arguments (nothing is launched when a check fails), encodes the
+// TMA tensor maps, carves the caller's workspace and enqueues the kernels on
+// the caller's stream.  It never allocates device memory and never
+// synchronises, except in strict-validation mode and in
+// mxfa_read_device_status, which are documented to.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+#include <string>
+#include <vector>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "mxfa.h"
+
+#include "common.cuh"
+#include "simt.cuh"
+#include "prefill_tc.cuh"
+#include "sched.cuh"
+
+using namespace mxfa;
+
+namespace {
+
+thread_local std::string g_err;
+thread_local uint32_t g_detail = 0;
+
+mxfa_status_t fail(mxfa_status_t s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+mxfa_status_t cuda_fail(cudaError_t e, const char *what) {
+  return fail(MXFA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define MXFA_CUDA(call)                               \
+  do {                                                \
+    cudaError_t e_ = (call);                          \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+bool strict_mode() {
+  static int v = [] {
+    const char *e = std::getenv("MXFA_STRICT_VALIDATION");
+    return (e && e[0] == '1') ? 1 : 0;
+  }();
+  return v != 0;
+}
+
+int elem_bytes(mxfa_dtype_t dt) { return dt == MXFA_F32 ? 4 : 2; }
+
+bool dtype_ok(int dt) { return dt == MXFA_F32 || dt == MXFA_F16 || dt == MXFA_BF16; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------- device facts
+std::mutex g_dev_mu;
+std::vector<int> g_sms;
+std::set<std::pair<const void *, int>> g_smem_set;
+
+mxfa_status_t sm_count(int *out) {
+  int dev = 0;
+  MXFA_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if ((int)g_sms.size() <= dev) g_sms.resize(dev + 1, 0);
+  if (g_sms[dev] == 0) MXFA_CUDA(cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev));
+  *out = g_sms[dev];
+  return MXFA_OK;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+mxfa_status_t ensure_smem(const void *kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return MXFA_OK;
+  int dev = 0;
+  MXFA_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_smem_set.count({kernel, dev})) return MXFA_OK;
+  MXFA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  g_smem_set.insert({kernel, dev});
+  return MXFA_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+mxfa_status_t get_encoder(EncodeTiledFn *fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!cached) return fail(MXFA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (%s)", cudaGetErrorString(err));
+  *fn = cached;
+  return MXFA_OK;
+}
+
+// 3-D map over [rows][heads][D] (16-bit elements), box = 128 rows x 1 head x
+// 64 columns, 128-byte swizzle; rows past `rows` read as zero.
+mxfa_status_t make_map(CUtensorMap *map, const void *base, mxfa_dtype_t dt, int D, int heads, int64_t rows,
+                       int64_t row_stride, int64_t head_stride) {
+  EncodeTiledFn enc;
+  mxfa_status_t st = get_encoder(&enc);
+  if (st != MXFA_OK) return st;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)head_stride * 2, (cuuint64_t)row_stride * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTcBlockM};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, dt == MXFA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                   const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MXFA_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MXFA_OK;
+}
+
+// ---------------------------------------------------------------- validation
+mxfa_status_t check_ptr(const void *p, const char *name, bool allow_null = false) {
+  if (!p) return allow_null ? MXFA_OK : fail(MXFA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(p) % 16) return fail(MXFA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return MXFA_OK;
+}
+
+mxfa_status_t check_stride(int64_t s, int eb, const char *name) {
+  if (s <= 0) return fail(MXFA_ERR_INVALID_ARG, "%s must be positive", name);
+  if ((s * eb) % 16) return fail(MXFA_ERR_INVALID_ARG, "%s (%lld elements) is not a multiple of 16 bytes", name,
+                                 (long long)s);
+  return MXFA_OK;
+}
+
+#define MXFA_TRY(x)                      \
+  do {                                   \
+    mxfa_status_t s_ = (x);              \
+    if (s_ != MXFA_OK) return s_;        \
+  } while (0)
+
+mxfa_status_t check_workspace(const void *ws, size_t have, size_t need) {
+  if (!ws) return fail(MXFA_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(MXFA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (have < need) return fail(MXFA_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", have, need);
+  return MXFA_OK;
+}
+
+// Strict mode: copy a cumulative-length array to the host and check it.
+mxfa_status_t strict_check_cu(const int32_t *cu, int batch, int total, int max_len, const char *name,
+                              cudaStream_t st) {
+  std::vector<int32_t> h(batch + 1);
+  MXFA_CUDA(cudaMemcpyAsync(h.data(), cu, sizeof(int32_t) * (batch + 1), cudaMemcpyDeviceToHost, st));
+  MXFA_CUDA(cudaStreamSynchronize(st));
+  if (h[0] != 0) return fail(MXFA_ERR_INVALID_ARG, "%s[0] = %d, expected 0", name, h[0]);
+  for (int b = 0; b < batch; ++b) {
+    const int len = h[b + 1] - h[b];
+    if (len < 0) return fail(MXFA_ERR_INVALID_ARG, "%s decreases at %d", name, b);
+    if (len > max_len) return fail(MXFA_ERR_INVALID_ARG, "%s: length %d of sequence %d exceeds the maximum %d", name,
+                                   len, b, max_len);
+  }
+  if (h[batch] != total) return fail(MXFA_ERR_INVALID_ARG, "%s[batch] = %d, expected the total %d", name, h[batch],
+                                     total);
+  return MXFA_OK;
+}
+
+float resolve_scale(float s, int dqk) { return std::isnan(s) ? 1.0f / std::sqrt((float)dqk) : s; }
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- launchers
+template <typename T, int DVL>
+mxfa_status_t launch_simt_dv(const AttnParams &p, dim3 grid, size_t smem, cudaStream_t st) {
+  auto k = attn_fwd_simt_kernel<T, DVL>;
+  MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(k), smem));
+  k<<<grid, kSimtWarps * 32, smem, st>>>(p);
+  MXFA_CUDA(cudaGetLastError());
+  return MXFA_OK;
+}
+
+template <typename T>
+mxfa_status_t launch_simt(const AttnParams &p, int max_rows_per_seq_head, cudaStream_t st) {
+  const size_t smem = simt_smem_bytes(p.dqk, p.dv);
+  const int G = p.hq / p.hkv;
+  dim3 grid((unsigned)((max_rows_per_seq_head * (int64_t)G + kSimtWarps - 1) / kSimtWarps), p.hkv, p.batch);
+  if (grid.x == 0) return MXFA_OK;
+  if (p.dv <= 64) return launch_simt_dv<T, 2>(p, grid, smem, st);
+  if (p.dv <= 128) return launch_simt_dv<T, 4>(p, grid, smem, st);
+  return launch_simt_dv<T, 16>(p, grid, smem, st);
+}
+
+mxfa_status_t launch_simt_any(mxfa_dtype_t dt, const AttnParams &p, int max_rows, cudaStream_t st) {
+  if (dt == MXFA_F32) return launch_simt<float>(p, max_rows, st);
+  if (dt == MXFA_BF16) return launch_simt<__nv_bfloat16>(p, max_rows, st);
+  return launch_simt<__half>(p, max_rows, st);
+}
+
+template <int D, bool BF16>
+mxfa_status_t launch_tc(const AttnParams &p, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                        cudaStream_t st) {
+  int sms = 0;
+  MXFA_TRY(sm_count(&sms));
+  auto k = attn_fwd_tc_kernel<D, BF16>;
+  MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(k), PrefillCfg<D>::kSmemBytes));
+  k<<<sms, kTcThreads, PrefillCfg<D>::kSmemBytes, st>>>(p, mq, mk, mv);
+  MXFA_CUDA(cudaGetLastError());
+  return MXFA_OK;
+}
+
+// Workspace layout of the varlen tensor-core prefill.
+struct VarlenWs {
+  size_t prefix, bucket, pairs, total;
+  int n_buckets, max_pairs;
+};
+VarlenWs varlen_ws(int batch, int max_sq, int max_sk) {
+  VarlenWs w;
+  w.n_buckets = 2 * ((max_sk + kTcBlockN - 1) / kTcBlockN) + 1;
+  w.max_pairs = batch * ((max_sq + kTcUnitRows - 1) / kTcUnitRows);
+  w.prefix = sizeof(WsHeader);
+  w.bucket = w.prefix + align256(sizeof(int) * (size_t)(batch + 1));
+  w.pairs = w.bucket + align256(sizeof(int) * (size_t)w.n_buckets);
+  w.total = w.pairs + align256(sizeof(int2) * (size_t)(w.max_pairs > 0 ? w.max_pairs : 1));
+  return w;
+}
+
+// Shared by the batched and varlen prefill entry points.
+mxfa_status_t prefill(AttnParams &p, mxfa_dtype_t dt, int D, bool varlen, int64_t rows_q, int64_t rows_k,
+                      void *ws, cudaStream_t st) {
+  const bool tc = dt != MXFA_F32 && (D == 64 || D == 128);
+  if (!tc) return launch_simt_any(dt, p, p.max_sq, st);
+  if (varlen) {
+    const VarlenWs w = varlen_ws(p.batch, p.max_sq, p.max_sk);
+    char *base = static_cast<char *>(ws);
+    int2 *pairs = reinterpret_cast<int2 *>(base + w.pairs);
+    prefill_prep_kernel<<<1, kPrepThreads, 0, st>>>(p, reinterpret_cast<int *>(base + w.prefix),
+                                                     reinterpret_cast<int *>(base + w.bucket), w.n_buckets, pairs,
+                                                     w.max_pairs);
+    MXFA_CUDA(cudaGetLastError());
+    p.pairs = pairs;
+  }
+  CUtensorMap mq, mk, mv;
+  MXFA_TRY(make_map(&mq, p.q, dt, D, p.hq, rows_q, p.q_rs, p.q_hs));
+  MXFA_TRY(make_map(&mk, p.k, dt, D, p.hkv, rows_k, p.k_rs, p.k_hs));
+  MXFA_TRY(make_map(&mv, p.v, dt, D, p.hkv, rows_k, p.v_rs, p.v_hs));
+  const bool bf = dt == MXFA_BF16;
+  if (D == 128) return bf ? launch_tc<128, true>(p, mq, mk, mv, st) : launch_tc<128, false>(p, mq, mk, mv, st);
+  return bf ? launch_tc<64, true>(p, mq, mk, mv, st) : launch_tc<64, false>(p, mq, mk, mv, st);
+}
+
+mxfa_status_t check_heads(int Hq, int Hkv) {
+  if (Hq <= 0 || Hkv <= 0) return fail(MXFA_ERR_INVALID_ARG, "head counts must be positive (Hq=%d, Hkv=%d)", Hq, Hkv);
+  if (Hq % Hkv) return fail(MXFA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  return MXFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mxfa_last_error(void) { return g_err.c_str(); }
+
+uint32_t mxfa_version(void) { return (0u << 16) | (1u << 8) | 0u; }
+
+uint32_t mxfa_device_status_detail(void) { return g_detail; }
+
+mxfa_status_t mxfa_read_device_status(const void *workspace, void *stream) {
+  if (!workspace) return fail(MXFA_ERR_WORKSPACE, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t h[2] = {0, 0};
+  MXFA_CUDA(cudaMemcpyAsync(h, workspace, sizeof h, cudaMemcpyDeviceToHost, st));
+  MXFA_CUDA(cudaStreamSynchronize(st));
+  g_detail = h[1];
+  if (h[0] != 0) {
+    MXFA_CUDA(cudaMemsetAsync(const_cast<void *>(workspace), 0, sizeof h, st));
+    MXFA_CUDA(cudaStreamSynchronize(st));
+    return fail(static_cast<mxfa_status_t>(h[0]), "device reported status %u at site 0x%x", h[0], h[1]);
+  }
+  return MXFA_OK;
+}
+
+size_t mxfa_attn_fwd_workspace_size(int, int, int, int, int, int, mxfa_dtype_t) { return sizeof(WsHeader); }
+
+size_t mxfa_attn_varlen_fwd_workspace_size(int batch, int max_seqlen_q, int max_seqlen_k, int, int D,
+                                           mxfa_dtype_t dtype) {
+  if (dtype == MXFA_F32 || (D != 64 && D != 128) || batch <= 0) return sizeof(WsHeader);
+  return varlen_ws(batch, max_seqlen_q, max_seqlen_k).total;
+}
+
+mxfa_status_t mxfa_attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Sq, int Sk,
+                            int Hq, int Hkv, int D, mxfa_dtype_t dtype, int64_t q_row_stride, int64_t q_head_stride,
+                            int64_t k_row_stride, int64_t k_head_stride, int64_t v_row_stride,
+                            int64_t v_head_stride, int64_t o_row_stride, int64_t o_head_stride, float softmax_scale,
+                            int causal, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!dtype_ok(dtype)) return fail(MXFA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (B < 0 || Sq < 0 || Sk < 0) return fail(MXFA_ERR_INVALID_ARG, "negative size (B=%d, Sq=%d, Sk=%d)", B, Sq, Sk);
+  MXFA_TRY(check_heads(Hq, Hkv));
+  if (D != 64 && D != 128) return fail(MXFA_ERR_UNSUPPORTED, "head dim %d is not supported (64 or 128)", D);
+  if (std::isinf(softmax_scale)) return fail(MXFA_ERR_INVALID_ARG, "softmax_scale is infinite");
+  if (B == 0 || Sq == 0) return MXFA_OK;
+  const int eb = elem_bytes(dtype);
+  MXFA_TRY(check_ptr(q, "q"));
+  MXFA_TRY(check_ptr(o, "o"));
+  MXFA_TRY(check_ptr(lse, "lse", true));
+  if (Sk > 0) {
+    MXFA_TRY(check_ptr(k, "k"));
+    MXFA_TRY(check_ptr(v, "v"));
+  }
+  MXFA_TRY(check_stride(q_row_stride, eb, "q_row_stride"));
+  MXFA_TRY(check_stride(q_head_stride, eb, "q_head_stride"));
+  MXFA_TRY(check_stride(k_row_stride, eb, "k_row_stride"));
+  MXFA_TRY(check_stride(k_head_stride, eb, "k_head_stride"));
+  MXFA_TRY(check_stride(v_row_stride, eb, "v_row_stride"));
+  MXFA_TRY(check_stride(v_head_stride, eb, "v_head_stride"));
+  MXFA_TRY(check_stride(o_row_stride, eb, "o_row_stride"));
+  MXFA_TRY(check_stride(o_head_stride, eb, "o_head_stride"));
+  const int64_t rows_q = (int64_t)B * Sq, rows_k = (int64_t)B * Sk;
+  if (rows_q > INT32_MAX || rows_k > INT32_MAX) return fail(MXFA_ERR_INVALID_ARG, "B*S exceeds 2^31 rows");
+  MXFA_TRY(check_workspace(workspace, workspace_bytes, mxfa_attn_fwd_workspace_size(B, Sq, Sk, Hq, Hkv, D, dtype)));
+
+  AttnParams p{};
+  p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+  p.cu_q = nullptr; p.cu_k = nullptr;
+  p.batch = B; p.sq = Sq; p.sk = Sk; p.max_sq = Sq; p.max_sk = Sk;
+  p.hq = Hq; p.hkv = Hkv; p.dqk = D; p.dv = D;
+  p.q_rs = q_row_stride; p.q_hs = q_head_stride; p.k_rs = k_row_stride; p.k_hs = k_head_stride;
+  p.v_rs = v_row_stride; p.v_hs = v_head_stride; p.o_rs = o_row_stride; p.o_hs = o_head_stride;
+  p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
+  p.causal = causal ? 1 : 0;
+  p.hdr = static_cast<WsHeader *>(workspace);
+  p.pairs = nullptr;
+  return prefill(p, dtype, D, false, rows_q, rows_k, workspace, static_cast<cudaStream_t>(stream));
+}
+
+mxfa_status_t mxfa_attn_varlen_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int batch, int total_q,
+                                   int total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int D,
+                                   mxfa_dtype_t dtype, float softmax_scale, int causal, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+  if (!dtype_ok(dtype)) return fail(MXFA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (batch < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
+    return fail(MXFA_ERR_INVALID_ARG, "negative size");
+  MXFA_TRY(check_heads(Hq, Hkv));
+  if (D != 64 && D != 128) return fail(MXFA_ERR_UNSUPPORTED, "head dim %d is not supported (64 or 128)", D);
+  if (std::isinf(softmax_scale)) return fail(MXFA_ERR_INVALID_ARG, "softmax_scale is infinite");
+  if (batch == 0 || total_q == 0) return MXFA_OK;
+  if (!cu_seqlens_q || !cu_seqlens_k) return fail(MXFA_ERR_INVALID_ARG, "cu_seqlens_q / cu_seqlens_k is NULL");
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return fail(MXFA_ERR_INVALID_ARG, "max_seqlen exceeds the total token count");
+  MXFA_TRY(check_ptr(q, "q"));
+  MXFA_TRY(check_ptr(o, "o"));
+  MXFA_TRY(check_ptr(lse, "lse", true));
+  if (total_k > 0) {
+    MXFA_TRY(check_ptr(k, "k"));
+    MXFA_TRY(check_ptr(v, "v"));
+  }
+  MXFA_TRY(check_workspace(workspace, workspace_bytes,
+                           mxfa_attn_varlen_fwd_workspace_size(batch, max_seqlen_q, max_seqlen_k, Hq, D, dtype)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (strict_mode()) {
+    MXFA_TRY(strict_check_cu(cu_seqlens_q, batch, total_q, max_seqlen_q, "cu_seqlens_q", st));
+    MXFA_TRY(strict_check_cu(cu_seqlens_k, batch, total_k, max_seqlen_k, "cu_seqlens_k", st));
+  }
+  AttnParams p{};
+  p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+  p.cu_q = cu_seqlens_q; p.cu_k = cu_seqlens_k;
+  p.batch = batch; p.sq = 0; p.sk = 0; p.max_sq = max_seqlen_q; p.max_sk = max_seqlen_k;
+  p.hq = Hq; p.hkv = Hkv; p.dqk = D; p.dv = D;
+  p.q_rs = (int64_t)Hq * D; p.q_hs = D; p.k_rs = (int64_t)Hkv * D; p.k_hs = D;
+  p.v_rs = (int64_t)Hkv * D; p.v_hs = D; p.o_rs = (int64_t)Hq * D; p.o_hs = D;
+  p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
+  p.causal = causal ? 1 : 0;
+  p.hdr = static_cast<WsHeader *>(workspace);
+  p.pairs = nullptr;
+  return prefill(p, dtype, D, true, total_q, total_k, workspace, st);
+}
+
+size_t mxfa_attn_decode_splitkv_workspace_size(int, int, int, int, int, int, mxfa_dtype_t) {
+  return sizeof(WsHeader);
+}
+
+mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
+                                       const int32_t *qo_indptr, const int32_t *kv_indptr, int batch, int total_q,
+                                       int total_kv, int max_q_len, int max_kv_len, int Hq, int Hkv, int Dqk, int Dv,
+                                       int64_t k_row_stride, int64_t v_row_stride, mxfa_dtype_t dtype,
+                                       float softmax_scale, int causal, int num_splits, void *workspace,
+                                       size_t workspace_bytes, void *stream) {
+  if (!dtype_ok(dtype)) return fail(MXFA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (batch < 0 || total_q < 0 || total_kv < 0 || max_q_len < 0 || max_kv_len < 0 || num_splits < 0)
+    return fail(MXFA_ERR_INVALID_ARG, "negative size");
+  MXFA_TRY(check_heads(Hq, Hkv));
+  const bool dims_ok = (Dqk == 64 && Dv == 64) || (Dqk == 128 && Dv == 128) || (Dqk == 576 && Dv == 512);
+  if (!dims_ok) return fail(MXFA_ERR_UNSUPPORTED, "(Dqk, Dv) = (%d, %d) is not supported", Dqk, Dv);
+  if (std::isinf(softmax_scale)) return fail(MXFA_ERR_INVALID_ARG, "softmax_scale is infinite");
+  if (batch == 0 || total_q == 0) return MXFA_OK;
+  if (!qo_indptr || !kv_indptr) return fail(MXFA_ERR_INVALID_ARG, "qo_indptr / kv_indptr is NULL");
+  if (max_q_len > total_q || max_kv_len > total_kv)
+    return fail(MXFA_ERR_INVALID_ARG, "max length exceeds the total count");
+  const int eb = elem_bytes(dtype);
+  MXFA_TRY(check_ptr(q, "q"));
+  MXFA_TRY(check_ptr(o, "o"));
+  MXFA_TRY(check_ptr(lse, "lse", true));
+  if (total_kv > 0) {
+    MXFA_TRY(check_ptr(k, "k"));
+    MXFA_TRY(check_ptr(v, "v"));
+    MXFA_TRY(check_stride(k_row_stride, eb, "k_row_stride"));
+    MXFA_TRY(check_stride(v_row_stride, eb, "v_row_stride"));
+    if (k_row_stride < (int64_t)Hkv * Dqk || v_row_stride < (int64_t)Hkv * Dv)
+      return fail(MXFA_ERR_INVALID_ARG, "row strides smaller than a row");
+  }
+  MXFA_TRY(check_workspace(workspace, workspace_bytes,
+                           mxfa_attn_decode_splitkv_workspace_size(batch, max_q_len, Hq, Dv, max_kv_len, num_splits,
+                                                                   dtype)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (strict_mode()) {
+    MXFA_TRY(strict_check_cu(qo_indptr, batch, total_q, max_q_len, "qo_indptr", st));
+    MXFA_TRY(strict_check_cu(kv_indptr, batch, total_kv, max_kv_len, "kv_indptr", st));
+  }
+  AttnParams p{};
+  p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+  p.cu_q = qo_indptr; p.cu_k = kv_indptr;
+  p.batch = batch; p.max_sq = max_q_len; p.max_sk = max_kv_len;
+  p.hq = Hq; p.hkv = Hkv; p.dqk = Dqk; p.dv = Dv;
+  p.q_rs = (int64_t)Hq * Dqk; p.q_hs = Dqk; p.k_rs = k_row_stride; p.k_hs = Dqk;
+  p.v_rs = v_row_stride; p.v_hs = Dv; p.o_rs = (int64_t)Hq * Dv; p.o_hs = Dv;
+  p.scale_log2 = resolve_scale(softmax_scale, Dqk) * kLog2e;
+  p.causal = causal ? 1 : 0;
+  p.hdr = static_cast<WsHeader *>(workspace);
+  p.pairs = nullptr;
+  return launch_simt_any(dtype, p, max_q_len, st);
+}
+
+}  // extern "C"

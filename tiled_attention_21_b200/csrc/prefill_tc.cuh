@@ -1,0 +1,487 @@
+// prefill_tc.cuh -- tensor-core attention forward for bf16 / f16 (sm_100a).
+//
+// One persistent CTA per SM walks a list of work units.  A unit is
+// (sequence b, 256-row query block m, query head h) and is processed as two
+// 128-row query tiles t = 0, 1 that share every K/V tile.  Per KV tile j
+// (128 keys) and query tile t:
+//     S_t  = Q_t K_j^T           tcgen05.mma, A = Q (smem), B = K (smem),
+//                                fp32 accumulator in TMEM
+//     P_t  = exp2(c*S_t - m)     softmax warpgroup t, one thread per row,
+//                                c = softmax_scale*log2(e); P written back
+//                                into TMEM over S_t as bf16/f16
+//     O_t += P_t V_j             tcgen05.mma, A = P (TMEM), B = V (smem)
+// The online-softmax bookkeeping follows mxflashattn 1.4.0 prefill.py
+// (prefill_chunked_reference: running max, correction of the accumulator,
+// running sum, rows with nothing visible end at O = 0) and oxillama-runtime
+// 0.1.0 flash_attention.rs (causal tile skipping), with one change of
+// schedule: the accumulator is only rescaled when a row's maximum grows by
+// more than 2^8.  Until then O and l keep the stale maximum as their common
+// base, which leaves O = acc / l and LSE = base + log2(l) exact.
+//
+// Roles (384 threads):
+//   warp 0      TMA producer: Q tiles once per unit, then K_j, V_j into a
+//               ring of shared-memory slots (128B-swizzled boxes of 64 cols)
+//   warp 1      TMEM allocator and single-thread MMA issuer; it alternates
+//               the two query tiles (PV_0(j), S_0(j+1), PV_1(j), S_1(j+1))
+//               so one tile's softmax overlaps the other tile's MMAs
+//   warps 4-7   softmax + epilogue of query tile 0 (TMEM lanes 0..127)
+//   warps 8-11  softmax + epilogue of query tile 1
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
+//
+// Every wait is bounded (see wait_bar); a wait that runs out records
+// MXFA_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag, and all
+// roles skip to the common teardown, which drains the TMA loads and MMAs
+// this CTA issued before TMEM is released.
+#pragma once
+
+#include <type_traits>
+
+#include "ptx.cuh"
+
+namespace mxfa {
+
+constexpr int kTcBlockM = 128;  // rows per query tile
+constexpr int kTcBlockN = 128;  // keys per KV tile
+constexpr int kTcUnitRows = 2 * kTcBlockM;
+constexpr int kTcThreads = 384;
+constexpr int kTcMaxSlots = 10;
+
+template <int D>
+struct PrefillCfg {
+  static constexpr int kAtoms = D / 64;                 // 128-byte column blocks per row
+  static constexpr int kAtomBytes = kTcBlockM * 128;    // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kTcBlockM * D * 2;  // one 128-row tile of Q, K or V
+  static constexpr int kSlots = D == 128 ? 5 : 10;
+  static constexpr int kCtrlBytes = 2048;               // barriers + slack to 1024-align the tiles
+  static constexpr int kSmemBytes = kCtrlBytes + (2 + kSlots) * kTileBytes;
+  static_assert(kSlots <= kTcMaxSlots, "slot count");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+struct PrefillCtrl {
+  uint64_t q_full, q_empty;
+  uint64_t slot_full[kTcMaxSlots], slot_empty[kTcMaxSlots];
+  uint64_t s_full[2], p_full[2], o_done[2], o_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Wait-site codes reported in the workspace on a timeout.
+enum : uint32_t {
+  kSiteQEmpty = 0x101, kSiteSlotEmpty, kSiteQFull, kSiteSlotFull, kSitePFull, kSiteOEmpty,
+  kSiteSFull, kSiteODone, kSiteDrain
+};
+
+struct UnitInfo {
+  int b, m, h, g;
+  SeqRange sr;
+  int n[2];  // KV tiles needed by query tile 0 / 1
+};
+
+// Unit u of the schedule.  Uniform lengths: 256-row blocks ordered by
+// decreasing causal cost (last block first), all sequences of a block
+// consecutively, heads innermost.  Varlen: the (b, m) pairs sorted by the
+// prep kernel.
+__device__ __forceinline__ UnitInfo unit_info(const AttnParams &p, int u) {
+  UnitInfo ui;
+  const int pr = u / p.hq;
+  ui.h = u - pr * p.hq;
+  ui.g = ui.h / (p.hq / p.hkv);
+  if (p.cu_q == nullptr) {
+    const int nblk = (p.sq + kTcUnitRows - 1) / kTcUnitRows;
+    ui.m = nblk - 1 - pr / p.batch;
+    ui.b = pr - (pr / p.batch) * p.batch;
+  } else {
+    const int2 pm = p.pairs[pr];
+    ui.b = pm.x;
+    ui.m = pm.y;
+  }
+  ui.sr = seq_range(p, ui.b);
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int first = ui.m * kTcUnitRows + t * kTcBlockM;
+    if (first >= ui.sr.sq) {
+      ui.n[t] = 0;
+    } else {
+      const int last = min(ui.sr.sq - 1, first + kTcBlockM - 1);
+      ui.n[t] = (visible_keys(last, ui.sr.sq, ui.sr.sk, p.causal) + kTcBlockN - 1) / kTcBlockN;
+    }
+  }
+  return ui;
+}
+
+// Snake walk of the sorted unit list: round r, CTA c takes unit
+// r*G + c (even r) or r*G + G-1-c (odd r).
+__device__ __forceinline__ int unit_of(int round, int cta, int grid) {
+  return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+}
+
+__device__ __forceinline__ int n_units_of(const AttnParams &p) {
+  if (p.cu_q == nullptr) return p.batch * ((p.sq + kTcUnitRows - 1) / kTcUnitRows) * p.hq;
+  return (int)(*reinterpret_cast<volatile uint32_t *>(&p.hdr->n_units)) * p.hq;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kTcThreads, 1)
+attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+  using Cfg = PrefillCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  PrefillCtrl *ctrl = reinterpret_cast<PrefillCtrl *>(smem_raw);
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t tiles_u32 = (raw_u32 + 1024u + 1023u) & ~1023u;
+  const uint32_t q_u32 = tiles_u32;                              // 2 query tiles
+  const uint32_t ring_u32 = tiles_u32 + 2 * Cfg::kTileBytes;     // kSlots KV slots
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int *abort_flag = &ctrl->abort;
+  WsHeader *hdr = p.hdr;
+
+  const uint32_t b_qf = smem_u32(&ctrl->q_full), b_qe = smem_u32(&ctrl->q_empty);
+  auto b_sf = [&](int s) { return smem_u32(&ctrl->slot_full[s]); };
+  auto b_se = [&](int s) { return smem_u32(&ctrl->slot_empty[s]); };
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_qf, 1);
+    mbar_init(b_qe, 1);
+    for (int s = 0; s < Cfg::kSlots; ++s) {
+      mbar_init(b_sf(s), 1);
+      mbar_init(b_se(s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(smem_u32(&ctrl->s_full[t]), 1);
+      mbar_init(smem_u32(&ctrl->p_full[t]), 4 * 32);
+      mbar_init(smem_u32(&ctrl->o_done[t]), 1);
+      mbar_init(smem_u32(&ctrl->o_empty[t]), 4 * 32);
+    }
+    mbar_init(smem_u32(&ctrl->drain), 1);
+    ctrl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctrl->tmem_base), 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+
+  const int n_units = n_units_of(p);
+  const int grid = gridDim.x, cta = blockIdx.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t ring = 0, q_issued = 0;
+      bool ok = true;
+      for (int it = 0, u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
+        const UnitInfo ui = unit_info(p, u);
+        const int nmax = max(ui.n[0], ui.n[1]);
+        if (it > 0 && !wait_bar(b_qe, (it - 1) & 1, abort_flag, hdr, kSiteQEmpty)) break;
+        mbar_arrive_expect_tx(b_qf, 2 * Cfg::kTileBytes);
+        const int qrow = ui.sr.q0 + ui.m * kTcUnitRows;
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int a = 0; a < Cfg::kAtoms; ++a)
+            tma_load_3d(q_u32 + t * Cfg::kTileBytes + a * Cfg::kAtomBytes, &tm_q, b_qf, a * 64, ui.h,
+                        qrow + t * kTcBlockM);
+        ++q_issued;
+        for (int j = 0; j < nmax && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv, ++ring) {
+            const int s = ring % Cfg::kSlots;
+            if (!wait_bar(b_se(s), ((ring / Cfg::kSlots) & 1) ^ 1, abort_flag, hdr, kSiteSlotEmpty)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(b_sf(s), Cfg::kTileBytes);
+            const CUtensorMap *tm = kv ? &tm_v : &tm_k;
+#pragma unroll
+            for (int a = 0; a < Cfg::kAtoms; ++a)
+              tma_load_3d(ring_u32 + s * Cfg::kTileBytes + a * Cfg::kAtomBytes, tm, b_sf(s), a * 64, ui.g,
+                          ui.sr.k0 + j * kTcBlockN);
+          }
+        }
+      }
+      // Teardown: every load this thread issued must have landed before the
+      // CTA exits (on the normal path they were all consumed already).
+      const uint64_t t0 = global_ns();
+      if (q_issued > 0)
+        while (!mbar_test(b_qf, (q_issued - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        }
+      for (int s = 0; s < Cfg::kSlots; ++s) {
+        const uint32_t uses = ring / Cfg::kSlots + ((uint32_t)s < ring % Cfg::kSlots ? 1u : 0u);
+        if (uses == 0) continue;
+        while (!mbar_test(b_sf(s), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc_f16(BF16, kTcBlockM, kTcBlockN, false, false);
+      constexpr uint32_t idesc_o = make_idesc_f16(BF16, kTcBlockM, D, false, true);
+      uint32_t ring = 0, p_cnt[2] = {0, 0}, o_uses[2] = {0, 0};
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t qa = q_u32 + t * Cfg::kTileBytes, ka = ring_u32 + slot * Cfg::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Cfg::kAtomBytes + (kk & 3) * 32;
+          mma_ss(tmem + t * kTcBlockN, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&ctrl->s_full[t]));
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+        const uint32_t va = ring_u32 + slot * Cfg::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTcBlockN / 16; ++kk) {
+          mma_ts(tmem + 2 * kTcBlockN + t * D, tmem + t * kTcBlockN + kk * 8,
+                 make_sdesc_sw128(va + kk * 16 * 128, Cfg::kAtomBytes, 1024), idesc_o, (acc || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&ctrl->o_done[t]));
+      };
+      int it = 0;
+      bool ok = true;
+      for (int u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
+        const UnitInfo ui = unit_info(p, u);
+        const int nmax = max(ui.n[0], ui.n[1]);
+        if (!wait_bar(b_qf, it & 1, abort_flag, hdr, kSiteQFull)) break;
+        tc_fence_after();
+        if (nmax == 0) {
+          mma_commit(b_qe);
+          continue;
+        }
+        // prologue: S_t(0)
+        {
+          const int ks = ring % Cfg::kSlots;
+          if (!wait_bar(b_sf(ks), (ring / Cfg::kSlots) & 1, abort_flag, hdr, kSiteSlotFull)) break;
+          ++ring;
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t)
+            if (ui.n[t] > 0) issue_s(t, ks);
+          mma_commit(b_se(ks));
+          if (nmax == 1) mma_commit(b_qe);
+        }
+        for (int j = 0; j < nmax && ok; ++j) {
+          const int vs = ring % Cfg::kSlots;
+          if (!wait_bar(b_sf(vs), (ring / Cfg::kSlots) & 1, abort_flag, hdr, kSiteSlotFull)) {
+            ok = false;
+            break;
+          }
+          ++ring;
+          tc_fence_after();
+          const bool has_next = j + 1 < nmax;
+          int ks = -1;
+          uint32_t kph = 0;
+          bool kwaited = false;
+          if (has_next) {
+            ks = ring % Cfg::kSlots;
+            kph = (ring / Cfg::kSlots) & 1;
+            ++ring;
+          }
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j >= ui.n[t]) continue;
+            if (!wait_bar(smem_u32(&ctrl->p_full[t]), p_cnt[t] & 1, abort_flag, hdr, kSitePFull)) {
+              ok = false;
+              break;
+            }
+            ++p_cnt[t];
+            if (j == 0 && o_uses[t] > 0 &&
+                !wait_bar(smem_u32(&ctrl->o_empty[t]), (o_uses[t] - 1) & 1, abort_flag, hdr, kSiteOEmpty)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(t, vs, j > 0);
+            if (j + 1 < ui.n[t]) {
+              if (!kwaited) {
+                if (!wait_bar(b_sf(ks), kph, abort_flag, hdr, kSiteSlotFull)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                kwaited = true;
+              }
+              issue_s(t, ks);
+            }
+          }
+          if (!ok) break;
+          mma_commit(b_se(vs));
+          if (has_next) mma_commit(b_se(ks));
+          if (j == nmax - 2) mma_commit(b_qe);
+        }
+        if (!ok) break;
+        for (int t = 0; t < 2; ++t)
+          if (ui.n[t] > 0) ++o_uses[t];
+      }
+      // Teardown: all MMAs issued by this thread complete before TMEM is freed.
+      mma_commit(smem_u32(&ctrl->drain));
+      const uint64_t t0 = global_ns();
+      while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < kWaitBudgetNs) {
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int t = (warp - 4) >> 2;
+    const int sub = warp & 3;
+    const int r = sub * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16);
+    const uint32_t s_col = t * kTcBlockN, o_col = 2 * kTcBlockN + t * D;
+    const float c = p.scale_log2;
+    const bool neg = c < 0.f;
+    const uint32_t b_s = smem_u32(&ctrl->s_full[t]), b_p = smem_u32(&ctrl->p_full[t]);
+    const uint32_t b_od = smem_u32(&ctrl->o_done[t]), b_oe = smem_u32(&ctrl->o_empty[t]);
+    uint32_t s_cnt = 0, pv_cnt = 0;
+    int it = 0;
+    bool ok = true;
+    for (int u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
+      const UnitInfo ui = unit_info(p, u);
+      const int n = ui.n[t];
+      const int i = ui.m * kTcUnitRows + t * kTcBlockM + r;
+      const bool valid = i < ui.sr.sq;
+      const int nv = valid ? visible_keys(i, ui.sr.sq, ui.sr.sk, p.causal) : 0;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        const bool got_s = wait_bar(b_s, s_cnt & 1, abort_flag, hdr, kSiteSFull);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, got_s)) {
+          ok = false;
+          break;
+        }
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld32(trow + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(trow + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(trow + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(trow + s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        const int lim = nv - j * kTcBlockN;  // keys [0, lim) of this tile are visible
+        const bool masked = lim < kTcBlockN;
+        float ext = -INFINITY;
+        if (!masked) {
+          if (!neg) {
+#pragma unroll
+            for (int q = 0; q < 128; ++q) ext = fmaxf(ext, __uint_as_float(sr[q]));
+          } else {
+#pragma unroll
+            for (int q = 0; q < 128; ++q) ext = fmaxf(ext, -__uint_as_float(sr[q]));
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 128; ++q) {
+            const float x = neg ? -__uint_as_float(sr[q]) : __uint_as_float(sr[q]);
+            ext = (q < lim) ? fmaxf(ext, x) : ext;
+          }
+        }
+        const float m_tile = (ext == -INFINITY) ? -INFINITY : (neg ? -ext : ext) * c;
+        const float m_new = fmaxf(m_used, m_tile);
+        float alpha = 1.f;
+        bool need = false;
+        if (m_used == -INFINITY) {
+          m_used = m_new;  // nothing accumulated yet
+        } else if (m_new > m_used + 8.f) {
+          alpha = ex2(m_used - m_new);
+          m_used = m_new;
+          need = true;
+        }
+        const float base = (m_used == -INFINITY) ? 0.f : m_used;
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = q * 32 + 2 * e;
+            float p0 = ex2(fmaf(__uint_as_float(sr[c0]), c, -base));
+            float p1 = ex2(fmaf(__uint_as_float(sr[c0 + 1]), c, -base));
+            if (masked) {
+              p0 = c0 < lim ? p0 : 0.f;
+              p1 = c0 + 1 < lim ? p1 : 0.f;
+            }
+            rs0 += p0;
+            rs1 += p1;
+            pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+          }
+          tmem_st16(trow + s_col + q * 16, pk);
+        }
+        tmem_wait_st();
+        l = l * alpha + (rs0 + rs1);
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // PV_t(j-1) is the latest accumulation into O_t; it must be done.
+          const bool got_o = wait_bar(b_od, (pv_cnt - 1) & 1, abort_flag, hdr, kSiteODone);
+          __syncwarp();
+          if (!__all_sync(0xffffffffu, got_o)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t ov[32];
+            tmem_ld32(trow + o_col + q * 32, ov);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(trow + o_col + q * 32, ov);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(b_p);
+        ++pv_cnt;
+      }
+      if (!ok) break;
+      using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+      T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(ui.sr.q0 + i) * p.o_rs + (int64_t)ui.h * p.o_hs;
+      if (n > 0) {
+        const bool got_o = wait_bar(b_od, (pv_cnt - 1) & 1, abort_flag, hdr, kSiteODone);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, got_o)) break;
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t ov[32];
+          tmem_ld32(trow + o_col + q * 32, ov);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a0 = __uint_as_float(ov[2 * e]) * inv, a1 = __uint_as_float(ov[2 * e + 1]) * inv;
+            pk[e] = BF16 ? pack_bf16x2(a0, a1) : pack_f16x2(a0, a1);
+          }
+          if (valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + q * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(b_oe);
+      } else if (valid) {
+        uint4 *dst = reinterpret_cast<uint4 *>(orow);
+#pragma unroll
+        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
+      }
+      if (valid && p.lse) {
+        p.lse[(int64_t)(ui.sr.q0 + i) * p.hq + ui.h] =
+            l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      }
+    }
+  }
+
+  __syncwarp();  // the single-lane roles rejoin their warps before the CTA barrier
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace mxfa

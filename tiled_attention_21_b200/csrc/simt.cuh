@@ -1,0 +1,128 @@
+// simt.cuh -- exact attention forward on the CUDA cores.
+//
+// The fp32 path (and the decode shapes the tensor-core kernels do not
+// cover): FFMA dot products, warp-shuffle row reductions, an online softmax
+// in the exp2 domain with the scale folded into scale*log2(e)
+// (kernelbot-amd-mixed-mla 588924: SM_SCALE_LOG2E; oxillama-runtime 0.1.0
+// flash_attention.rs, flash_attention: tile max, correction factor, running
+// sum, normalise once at the end).
+//
+// Work split: a block of kSimtWarps warps serves kSimtWarps "rows" of one
+// (sequence, kv head); row r of the block is query token r / G and q head
+// g*G + r % G, so all of them read the same K/V tiles (the row flattening
+// of kernelbot-amd-mixed-mla 588924, _flash_fused: m = q_idx*heads + head).
+// One warp owns one row.  Keys are processed in tiles of 32, staged in
+// shared memory as fp32 (K rows padded by one word so the 32 lanes, one key
+// each, hit 32 different banks).  Lane l scores key l of the tile; for P.V
+// lane l owns output columns l, l+32, ...
+#pragma once
+
+#include "common.cuh"
+
+namespace mxfa {
+
+constexpr int kSimtWarps = 8;
+constexpr int kSimtKeys = 32;
+
+__host__ __device__ inline size_t simt_smem_bytes(int dqk, int dv) {
+  return sizeof(float) * ((size_t)kSimtWarps * dqk + (size_t)kSimtKeys * (dqk + 1) + (size_t)kSimtKeys * dv);
+}
+
+template <typename T, int DV_PER_LANE>
+__global__ void __launch_bounds__(kSimtWarps * 32)
+attn_fwd_simt_kernel(const AttnParams p) {
+  extern __shared__ float smem[];
+  const int dqk = p.dqk, dv = p.dv;
+  float *qs = smem;                                   // [kSimtWarps][dqk]
+  float *ks = qs + kSimtWarps * dqk;                  // [kSimtKeys][dqk + 1]
+  float *vs = ks + kSimtKeys * (dqk + 1);             // [kSimtKeys][dv]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.z, g = blockIdx.y;
+  const SeqRange sr = seq_range(p, b);
+  const int G = p.hq / p.hkv;
+  const int row = blockIdx.x * kSimtWarps + warp;    // flattened (query, head-in-group)
+  const int n_rows = sr.sq * G;
+  if (blockIdx.x * kSimtWarps >= n_rows) return;     // whole block idle (uniform)
+
+  const bool active = row < n_rows;
+  const int i = active ? row / G : 0;
+  const int h = g * G + (active ? row % G : 0);
+  const int n_vis = active ? visible_keys(i, sr.sq, sr.sk, p.causal) : 0;
+
+  // Keys the block needs: the largest visible count over its rows.
+  const int last_row = min(n_rows, (int)(blockIdx.x + 1) * kSimtWarps) - 1;
+  const int block_keys = visible_keys(last_row / G, sr.sq, sr.sk, p.causal);
+
+  const T *qrow = reinterpret_cast<const T *>(p.q) + (int64_t)(sr.q0 + i) * p.q_rs + (int64_t)h * p.q_hs;
+  for (int d = lane; d < dqk; d += 32) qs[warp * dqk + d] = active ? to_f32(qrow[d]) : 0.f;
+
+  float m = -INFINITY, l = 0.f;
+  float acc[DV_PER_LANE];
+#pragma unroll
+  for (int e = 0; e < DV_PER_LANE; ++e) acc[e] = 0.f;
+
+  const T *kbase = reinterpret_cast<const T *>(p.k) + (int64_t)g * p.k_hs;
+  const T *vbase = reinterpret_cast<const T *>(p.v) + (int64_t)g * p.v_hs;
+
+  for (int t0 = 0; t0 < block_keys; t0 += kSimtKeys) {
+    __syncthreads();  // previous tile fully consumed (also orders the qs writes)
+    const int nk = min(kSimtKeys, block_keys - t0);
+    for (int idx = threadIdx.x; idx < kSimtKeys * dqk; idx += blockDim.x) {
+      int j = idx / dqk, d = idx - j * dqk;
+      ks[j * (dqk + 1) + d] = j < nk ? to_f32(kbase[(int64_t)(sr.k0 + t0 + j) * p.k_rs + d]) : 0.f;
+    }
+    for (int idx = threadIdx.x; idx < kSimtKeys * dv; idx += blockDim.x) {
+      int j = idx / dv, d = idx - j * dv;
+      vs[j * dv + d] = j < nk ? to_f32(vbase[(int64_t)(sr.k0 + t0 + j) * p.v_rs + d]) : 0.f;
+    }
+    __syncthreads();
+    if (!active || t0 >= n_vis) continue;
+
+    // score of key t0 + lane, in the log2 domain
+    float s = 0.f;
+    const float *kr = ks + lane * (dqk + 1);
+    const float *qr = qs + warp * dqk;
+    for (int d = 0; d < dqk; ++d) s = fmaf(qr[d], kr[d], s);
+    float x = (t0 + lane < n_vis) ? s * p.scale_log2 : -INFINITY;
+
+    float tmax = x;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
+    const float m_new = fmaxf(m, tmax);
+    const float base = (m_new == -INFINITY) ? 0.f : m_new;   // all-masked guard
+    const float alpha = exp2f(m - base);                       // 0 when m = -inf
+    const float pj = exp2f(x - base);                          // 0 for masked keys
+    float psum = pj;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
+    l = l * alpha + psum;
+    m = m_new;
+#pragma unroll
+    for (int e = 0; e < DV_PER_LANE; ++e) acc[e] *= alpha;
+    for (int j = 0; j < nk; ++j) {
+      const float pb = __shfl_sync(0xffffffffu, pj, j);
+      const float *vr = vs + j * dv;
+#pragma unroll
+      for (int e = 0; e < DV_PER_LANE; ++e) {
+        const int d = lane + 32 * e;
+        if (d < dv) acc[e] = fmaf(pb, vr[d], acc[e]);
+      }
+    }
+  }
+  if (!active) return;
+
+  T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(sr.q0 + i) * p.o_rs + (int64_t)h * p.o_hs;
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+  for (int e = 0; e < DV_PER_LANE; ++e) {
+    const int d = lane + 32 * e;
+    if (d < dv) orow[d] = from_f32<T>(acc[e] * inv);
+  }
+  if (p.lse && lane == 0) {
+    const float lse = l > 0.f ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    p.lse[(int64_t)(sr.q0 + i) * p.hq + h] = lse;
+  }
+}
+
+}  // namespace mxfa
