@@ -353,7 +353,8 @@ def main():
                            "flops_per_step": flops, "l2": "flushed before every step (512 MiB write)",
                            "parallelism": f"replicas x{world}"},
                 "roofline": roofline, "cpu_baseline": cpu,
-                "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "e2e": None if args.only else {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                                               "d2h_bytes_per_step": d2h},
                 "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode}
         print(json.dumps(line), flush=True)
     if world > 1:
