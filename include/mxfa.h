@@ -114,6 +114,31 @@ mxfa_status_t mxfa_attn_varlen_fwd(const void *q, const void *k, const void *v, 
                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * mxfa_attn_varlen_fwd without a workspace argument.  The pages have no
+ * counterpart: this exists for callers that cannot allocate device memory
+ * when they run attention (plugins and services that plan all device memory
+ * up front, or code without access to the allocator that owns the device).
+ * Same arguments, layouts and results as mxfa_attn_varlen_fwd.
+ *   - Scratch: the schedule lives in a 1 MiB array owned by the library,
+ *     which every GPU that loads the library holds until the process exits.
+ *     A problem whose schedule needs more (mxfa_attn_varlen_fwd_workspace_size
+ *     above 1 MiB, e.g. very large batch x max_seqlen_q) is rejected with
+ *     MXFA_ERR_WORKSPACE and nothing is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Calls share the one array: calls that overlap on the GPU (different
+ *     streams without ordering, or several host threads) race and must not
+ *     be issued; order them on one stream.
+ *   - No device memory is allocated or freed.
+ */
+mxfa_status_t mxfa_attn_varlen_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                                           const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                           int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                                           int Hq, int Hkv, int D, mxfa_dtype_t dtype,
+                                           float softmax_scale, int causal, void *stream);
+
+/*
  * Split-KV decode (few queries per sequence, long KV), with the partial
  * (accumulator, max, sum) combine of kernelbot-amd-mixed-mla submission
  * 588924 (_flash_splitk / _reduce_splitk).

@@ -444,3 +444,67 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Varlen forward without a caller workspace.
+//
+// Some callers have no way to allocate device memory at the point where they
+// run attention: engine plugins and services that plan every device byte up
+// front and forbid allocation afterwards, or code that holds raw pointers but
+// no handle to the framework allocator that owns the device.  This entry point
+// serves them: the schedule the varlen path needs lives in a fixed scratch
+// array that belongs to the library, so the call allocates nothing.
+//
+// The array is a file-scope __device__ object: every GPU that loads this
+// library holds kNoAllocScratchBytes for it until the process exits.  Its name
+// is only a host-side stand-in in host code, so the device address is fetched
+// with cudaGetSymbolAddress once per device (with that device current) on the
+// first call there, and cached.
+// ---------------------------------------------------------------------------
+static constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+mxfa_status_t noalloc_scratch(void **out) {
+  int dev = 0;
+  MXFA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(MXFA_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MXFA_OK;
+}
+}  // namespace
+
+extern "C" mxfa_status_t mxfa_attn_varlen_fwd_noalloc(const void *q, const void *k, const void *v, void *o,
+                                                      float *lse, const int32_t *cu_seqlens_q,
+                                                      const int32_t *cu_seqlens_k, int batch, int total_q,
+                                                      int total_k, int max_seqlen_q, int max_seqlen_k, int Hq,
+                                                      int Hkv, int D, mxfa_dtype_t dtype, float softmax_scale,
+                                                      int causal, void *stream) {
+  if (!dtype_ok(dtype)) return fail(MXFA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (batch < 0 || max_seqlen_q < 0 || max_seqlen_k < 0) return fail(MXFA_ERR_INVALID_ARG, "negative size");
+  const size_t need = mxfa_attn_varlen_fwd_workspace_size(batch, max_seqlen_q, max_seqlen_k, Hq, D, dtype);
+  if (need > kNoAllocScratchBytes)
+    return fail(MXFA_ERR_WORKSPACE,
+                "this problem needs %zu bytes of scratch but the no-allocation entry point holds %zu; "
+                "call mxfa_attn_varlen_fwd with a workspace instead",
+                need, kNoAllocScratchBytes);
+  void *scratch = nullptr;
+  MXFA_TRY(noalloc_scratch(&scratch));
+  // The header (status word, unit count) must start at zero; the schedule
+  // tables after it are fully rewritten by every call.
+  MXFA_CUDA(cudaMemsetAsync(scratch, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
+  return mxfa_attn_varlen_fwd(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                              max_seqlen_k, Hq, Hkv, D, dtype, softmax_scale, causal, scratch, kNoAllocScratchBytes,
+                              stream);
+}
