@@ -1,0 +1,524 @@
+// decode_tc.cuh -- split-KV MLA decode on the tensor cores (sm_100a).
+//
+// Shape (kernelbot-amd-mixed-mla submission 588924, _flash_fused /
+// _flash_splitk / _reduce_splitk): every sequence b has q_len queries of Hq
+// heads that all read one shared latent KV row of 576 columns; the value is
+// the first 512 columns of that same row.  The q_len*Hq <= 64 query rows of a
+// sequence are flattened r = q*Hq + h and form the M = 64 side of every MMA.
+//
+// The KV cache is streamed exactly once: 64-key tiles arrive by TMA as nine
+// 8 KB column chunks (64 keys x 64 columns, 128B swizzle) into an 18-slot
+// ring (two tiles).  Each tile is used twice while resident:
+//     S   = Q K^T   tcgen05.mma M=64 N=64, 9 chunks x 4 K-steps, A = Q (smem)
+//     O  += P V     tcgen05.mma M=64 N=256 (x2), A = P (smem), B = chunks 0-7
+// S lives in TMEM lanes 16-31 of each sub-partition (double-buffered), O in
+// lanes 0-15 (all 512 columns): the two M=64 accumulators interleave in
+// TMEM.  A softmax warpgroup (128 threads) gives each query row two threads,
+// one per 32-key half of the tile (16-lane TMEM accesses), with the online
+// softmax of the prefill kernel (exp2 domain, rescale of O only when the
+// row max grows by more than 2^8).
+//
+// Work split (d1): the KV tiles of all sequences form one sequence of T
+// tiles; CTA c of G owns tiles [c*T/G, (c+1)*T/G) (automatic split), or each
+// sequence is cut into k near-equal pieces (num_splits = k) and a piece
+// belongs to the CTA whose range holds its first tile.  A sequence covered by
+// one piece is normalised and stored directly; otherwise every piece writes
+// its unnormalised partial (acc, running max, running sum) and
+// decode_combine_kernel merges them with weights 2^(m_s - max_s m_s).
+#pragma once
+
+#include <type_traits>
+
+#include <cub/block/block_scan.cuh>
+
+#include "ptx.cuh"
+
+namespace mxfa {
+
+constexpr int kDcRows = 64;       // M: query rows per sequence
+constexpr int kDcKeys = 64;       // keys per tile
+constexpr int kDcDqk = 576, kDcDv = 512;
+constexpr int kDcChunks = kDcDqk / 64;  // 9 column chunks per KV tile
+constexpr int kDcChunkBytes = kDcKeys * 128;
+constexpr int kDcSlots = 2 * kDcChunks;
+constexpr int kDcThreads = 256;
+constexpr int kDcCtrlBytes = 2048;
+constexpr int kDcSmemBytes = kDcCtrlBytes + (kDcChunks + kDcSlots) * kDcChunkBytes + kDcRows * 128;
+static_assert(kDcSmemBytes <= 232448, "shared memory budget");
+constexpr int kDcMaxGrid = 256;
+
+struct DecodeSched {
+  int *n_tiles;    // [batch] KV tiles per sequence
+  int *tile_pre;   // [batch + 1] prefix of n_tiles
+  int *seg_base;   // [batch + 1] first segment of each sequence
+  int *seg_cnt;    // [batch]
+  int4 *segs;      // [max_segs] (b, first tile, end tile, global first tile)
+  float *part_acc; // [max_segs][64][512]
+  float2 *part_ml; // [max_segs][64] (running max in log2 units, running sum)
+  int max_segs;
+  int num_splits;  // 0 = automatic
+  int grid;
+};
+
+struct DecodeCtrl {
+  uint64_t q_full, q_empty;
+  uint64_t slot_full[kDcSlots], slot_empty[kDcSlots];
+  uint64_t s_full[2], p_full, o_done, o_empty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+enum : uint32_t {
+  kDSiteQEmpty = 0x301, kDSiteSlotEmpty, kDSiteQFull, kDSiteSlotFull, kDSitePFull, kDSiteOEmpty, kDSiteSFull,
+  kDSiteODone
+};
+
+__device__ __forceinline__ int dc_range_start(int c, int T, int G) { return (int)(((int64_t)c * T) / G); }
+
+// First segment whose first global tile is >= x.
+__device__ __forceinline__ int dc_lower_bound(const int4 *segs, int n, int x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (segs[mid].w < x) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// ----------------------------------------------------------------------------
+// Schedule: one 1024-thread CTA.
+__global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, DecodeSched s) {
+  using Scan = cub::BlockScan<int, 1024>;
+  __shared__ typename Scan::TempStorage tmp;
+  __shared__ int carry;
+  const int tid = threadIdx.x, B = p.batch, G = s.grid;
+  // tiles per sequence and their prefix
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < B; base += 1024) {
+    const int b = base + tid;
+    int n = 0;
+    if (b < B) {
+      n = (p.cu_k[b + 1] - p.cu_k[b] + kDcKeys - 1) / kDcKeys;
+      if (p.cu_q[b + 1] - p.cu_q[b] <= 0) n = 0;  // no queries: nothing to compute
+      s.n_tiles[b] = n;
+    }
+    int incl, total;
+    Scan(tmp).InclusiveSum(n, incl, total);
+    if (b < B) s.tile_pre[b + 1] = carry + incl;
+    __syncthreads();
+    if (tid == 0) carry += total;
+    __syncthreads();
+  }
+  if (tid == 0) s.tile_pre[0] = 0;
+  const int T = carry;
+  __syncthreads();
+  // pieces per sequence
+  auto pieces = [&](int b) -> int {
+    const int n = s.n_tiles[b];
+    if (n == 0) return 0;
+    if (s.num_splits > 0) return min(s.num_splits, n);
+    const int P = s.tile_pre[b];
+    int cuts = 0;
+    for (int c = 1; c < G; ++c) {
+      const int x = dc_range_start(c, T, G);
+      // distinct boundaries strictly inside the sequence's tile range
+      cuts += (x > P && x < P + n && x != dc_range_start(c - 1, T, G)) ? 1 : 0;
+    }
+    return 1 + cuts;
+  };
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < B; base += 1024) {
+    const int b = base + tid;
+    const int k = b < B ? pieces(b) : 0;
+    if (b < B) s.seg_cnt[b] = k;
+    int incl, total;
+    Scan(tmp).InclusiveSum(k, incl, total);
+    if (b < B) s.seg_base[b] = carry + incl - k;
+    __syncthreads();
+    if (tid == 0) carry += total;
+    __syncthreads();
+  }
+  const int n_segs = carry;
+  if (tid == 0) s.seg_base[B] = n_segs;
+  __syncthreads();
+  // the pieces themselves
+  for (int b = tid; b < B; b += 1024) {
+    const int n = s.n_tiles[b], P = s.tile_pre[b], k = s.seg_cnt[b];
+    int idx = s.seg_base[b];
+    if (k == 0) continue;
+    if (s.num_splits > 0) {
+      for (int i = 0; i < k; ++i) {
+        const int t0 = (int)(((int64_t)i * n) / k), t1 = (int)(((int64_t)(i + 1) * n) / k);
+        if (idx < s.max_segs) s.segs[idx] = make_int4(b, t0, t1, P + t0);
+        ++idx;
+      }
+    } else {
+      int t0 = 0;
+      for (int c = 1; c <= G; ++c) {
+        const int x = c < G ? dc_range_start(c, T, G) : P + n;
+        if (x > P + t0 && x < P + n) {
+          if (idx < s.max_segs) s.segs[idx] = make_int4(b, t0, x - P, P + t0);
+          ++idx;
+          t0 = x - P;
+        }
+      }
+      if (idx < s.max_segs) s.segs[idx] = make_int4(b, t0, n, P + t0);
+    }
+  }
+  if (tid == 0) {
+    p.hdr->n_units = (uint32_t)min(n_segs, s.max_segs);
+    p.hdr->n_aux = (uint32_t)T;
+    if (n_segs > s.max_segs) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x401);
+  }
+}
+
+// ----------------------------------------------------------------------------
+template <bool BF16>
+__global__ void __launch_bounds__(kDcThreads, 1)
+attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
+                      const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv) {
+  extern __shared__ uint8_t smem_raw[];
+  DecodeCtrl *ctrl = reinterpret_cast<DecodeCtrl *>(smem_raw);
+  const uint32_t tiles_u32 = (smem_u32(smem_raw) + 1024u + 1023u) & ~1023u;
+  const uint32_t q_u32 = tiles_u32;                                  // 9 chunks of Q
+  const uint32_t ring_u32 = q_u32 + kDcChunks * kDcChunkBytes;       // 18 KV chunk slots
+  const uint32_t p_u32 = ring_u32 + kDcSlots * kDcChunkBytes;        // P: 64 rows x 128 B
+  uint8_t *p_gen = smem_raw + (p_u32 - smem_u32(smem_raw));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int *abort_flag = &ctrl->abort;
+  WsHeader *hdr = p.hdr;
+  auto b_sf = [&](int x) { return smem_u32(&ctrl->slot_full[x]); };
+  auto b_se = [&](int x) { return smem_u32(&ctrl->slot_empty[x]); };
+  const uint32_t b_qf = smem_u32(&ctrl->q_full), b_qe = smem_u32(&ctrl->q_empty);
+  const uint32_t b_pf = smem_u32(&ctrl->p_full), b_od = smem_u32(&ctrl->o_done), b_oe = smem_u32(&ctrl->o_empty);
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_qf, 1);
+    mbar_init(b_qe, 1);
+    for (int x = 0; x < kDcSlots; ++x) {
+      mbar_init(b_sf(x), 1);
+      mbar_init(b_se(x), 1);
+    }
+    mbar_init(smem_u32(&ctrl->s_full[0]), 1);
+    mbar_init(smem_u32(&ctrl->s_full[1]), 1);
+    mbar_init(b_pf, 128);
+    mbar_init(b_od, 1);
+    mbar_init(b_oe, 128);
+    mbar_init(smem_u32(&ctrl->drain), 1);
+    ctrl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kv);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctrl->tmem_base), 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+
+  // This CTA's pieces: those whose first tile lies in its tile range.
+  const int n_segs = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_units);
+  const int T = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_aux);
+  const int seg_lo = dc_lower_bound(s.segs, n_segs, dc_range_start(blockIdx.x, T, gridDim.x));
+  const int seg_hi = dc_lower_bound(s.segs, n_segs, dc_range_start(blockIdx.x + 1, T, gridDim.x));
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t ring = 0, q_issued = 0;
+      bool ok = true;
+      for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
+        const int4 sd = s.segs[sg];
+        const int q0 = p.cu_q[sd.x], k0 = p.cu_k[sd.x];
+        if (q_issued > 0 && !wait_bar(b_qe, (q_issued - 1) & 1, abort_flag, hdr, kDSiteQEmpty)) break;
+        mbar_arrive_expect_tx(b_qf, kDcChunks * kDcChunkBytes);
+        for (int c = 0; c < kDcChunks; ++c)
+          tma_load_2d(q_u32 + c * kDcChunkBytes, &tm_q, b_qf, c * 64, q0 * p.hq);
+        ++q_issued;
+        for (int j = sd.y; ok && j < sd.z; ++j) {
+          for (int c = 0; c < kDcChunks; ++c, ++ring) {
+            const int x = ring % kDcSlots;
+            if (!wait_bar(b_se(x), ((ring / kDcSlots) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(b_sf(x), kDcChunkBytes);
+            tma_load_2d(ring_u32 + x * kDcChunkBytes, &tm_kv, b_sf(x), c * 64, k0 + j * kDcKeys);
+          }
+        }
+      }
+      const uint64_t t0 = global_ns();
+      if (q_issued > 0)
+        while (!mbar_test(b_qf, (q_issued - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        }
+      for (int x = 0; x < kDcSlots; ++x) {
+        const uint32_t uses = ring / kDcSlots + ((uint32_t)x < ring % kDcSlots ? 1u : 0u);
+        if (uses == 0) continue;
+        while (!mbar_test(b_sf(x), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc_f16(BF16, kDcRows, kDcKeys, false, false);
+      constexpr uint32_t idesc_o = make_idesc_f16(BF16, kDcRows, 256, false, true);
+      const uint32_t s_tmem = tmem + (16u << 16);  // S: lanes 16-31 of each sub-partition
+      uint32_t ring = 0, g = 0, o_uses = 0;
+      bool ok = true;
+      // S(tile) into buffer buf; the tile's chunks start at ring slot `first`.
+      auto issue_s = [&](uint32_t buf, uint32_t first) -> bool {
+        for (int c = 0; c < kDcChunks; ++c) {
+          const uint32_t x = (first + c) % kDcSlots;
+          if (!wait_bar(b_sf(x), ((first + c) / kDcSlots) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(s_tmem + buf * kDcKeys, make_sdesc_sw128(q_u32 + c * kDcChunkBytes + kk * 32, 16, 1024),
+                   make_sdesc_sw128(ring_u32 + x * kDcChunkBytes + kk * 32, 16, 1024), idesc_s,
+                   (c > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(smem_u32(&ctrl->s_full[buf]));
+        mma_commit(b_se((first + kDcChunks - 1) % kDcSlots));  // the rope chunk is only read by S
+        return true;
+      };
+      for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
+        const int4 sd = s.segs[sg];
+        const int n = sd.z - sd.y;
+        if (!wait_bar(b_qf, (sg - seg_lo) & 1, abort_flag, hdr, kDSiteQFull)) break;
+        tc_fence_after();
+        if (!issue_s(g & 1, ring)) break;
+        if (n == 1) mma_commit(b_qe);
+        for (int jj = 0; jj < n; ++jj, ++g) {
+          const uint32_t first = ring;
+          ring += kDcChunks;
+          if (jj + 1 < n) {
+            if (!issue_s((g + 1) & 1, ring)) {
+              ok = false;
+              break;
+            }
+            if (jj + 2 == n) mma_commit(b_qe);
+          }
+          if (!wait_bar(b_pf, g & 1, abort_flag, hdr, kDSitePFull)) {
+            ok = false;
+            break;
+          }
+          if (jj == 0 && o_uses > 0 && !wait_bar(b_oe, (o_uses - 1) & 1, abort_flag, hdr, kDSiteOEmpty)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t vfirst = (first + half * 4) % kDcSlots;  // chunks 4*half..4*half+3 are consecutive
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tmem + half * 256, make_sdesc_sw128(p_u32 + kk * 32, 16, 1024),
+                     make_sdesc_sw128(ring_u32 + vfirst * kDcChunkBytes + kk * 16 * 128, kDcChunkBytes, 1024),
+                     idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(b_od);
+          for (int c = 0; c < kDcChunks - 1; ++c) mma_commit(b_se((first + c) % kDcSlots));
+        }
+        ++o_uses;
+      }
+      mma_commit(smem_u32(&ctrl->drain));
+      const uint64_t t0 = global_ns();
+      while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < kWaitBudgetNs) {
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int sub = warp & 3, half = lane >> 4;
+    const int r = sub * 16 + (lane & 15);                    // query row of this thread
+    const uint32_t o_row = tmem + ((uint32_t)(sub * 32) << 16);
+    const uint32_t s_row = tmem + ((uint32_t)(sub * 32 + 16) << 16);
+    const float c = p.scale_log2;
+    const bool neg = c < 0.f;
+    uint32_t g = 0;
+    bool ok = true;
+    for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
+      const int4 sd = s.segs[sg];
+      const int b = sd.x;
+      const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0, sk = p.cu_k[b + 1] - p.cu_k[b];
+      const int rows = sq * p.hq;
+      const bool valid = r < rows;
+      const int nv = valid ? visible_keys(r / p.hq, sq, sk, p.causal) : 0;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = sd.y; j < sd.z; ++j, ++g) {
+        const bool got = wait_bar(smem_u32(&ctrl->s_full[g & 1]), (g >> 1) & 1, abort_flag, hdr, kDSiteSFull);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[32];
+        tmem_ld_half32(s_row + (g & 1) * kDcKeys, sv);
+        const int lim = nv - j * kDcKeys - half * 32;  // keys [0, lim) of this half are visible
+        float ext = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float x = neg ? -__uint_as_float(sv[e]) : __uint_as_float(sv[e]);
+          ext = (e < lim) ? fmaxf(ext, x) : ext;
+        }
+        ext = fmaxf(ext, __shfl_xor_sync(0xffffffffu, ext, 16));
+        const float m_tile = (ext == -INFINITY) ? -INFINITY : (neg ? -ext : ext) * c;
+        const float m_new = fmaxf(m_used, m_tile);
+        float alpha = 1.f;
+        bool need = false;
+        if (m_used == -INFINITY) {
+          m_used = m_new;
+        } else if (m_new > m_used + 8.f) {
+          alpha = ex2(m_used - m_new);
+          m_used = m_new;
+          need = true;
+        }
+        const float base = (m_used == -INFINITY) ? 0.f : m_used;
+        uint32_t pk[16];
+        float rs = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), c, -base));
+          float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, -base));
+          p0 = (2 * e < lim) ? p0 : 0.f;
+          p1 = (2 * e + 1 < lim) ? p1 : 0.f;
+          rs += p0 + p1;
+          pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+        }
+        l = l * alpha + rs;
+        // P (single buffer) and O may be touched only once the previous P.V is done.
+        if (g > 0) {
+          const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone);
+          __syncwarp();
+          if (!__all_sync(0xffffffffu, got_o)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        if (j > sd.y && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int q = 0; q < kDcDv / 64; ++q) {
+            uint32_t ov[32];
+            tmem_ld_half32(o_row + q * 64, ov);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st_half32(o_row + q * 64, ov);
+          }
+          tmem_wait_st();
+        }
+        // P row r, keys half*32 .. half*32+31: four 16-byte chunks, 128B swizzle.
+        uint8_t *prow = p_gen + r * 128;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int chunk = (half * 4 + i) ^ (r & 7);
+          *reinterpret_cast<uint4 *>(prow + chunk * 16) = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(b_pf);
+      }
+      if (!ok) break;
+      // ---------------- epilogue of this piece
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      if (sd.z > sd.y) {
+        const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, got_o)) break;
+        tc_fence_after();
+      }
+      const bool direct = s.seg_cnt[b] == 1;
+      const int tok = q0 + (valid ? r / p.hq : 0), h = valid ? r % p.hq : 0;
+      using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+      for (int q = 0; q < kDcDv / 64; ++q) {
+        uint32_t ov[32];
+        tmem_ld_half32(o_row + q * 64, ov);
+        const int col = q * 64 + half * 32;
+        if (!valid) continue;
+        if (direct) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = BF16 ? pack_bf16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv)
+                         : pack_f16x2(__uint_as_float(ov[2 * e]) * inv, __uint_as_float(ov[2 * e + 1]) * inv);
+          T *orow = reinterpret_cast<T *>(p.o) + (int64_t)tok * p.o_rs + (int64_t)h * p.o_hs + col;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            reinterpret_cast<uint4 *>(orow)[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        } else {
+          float4 *dst = reinterpret_cast<float4 *>(s.part_acc + ((int64_t)sg * kDcRows + r) * kDcDv + col);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
+                                 __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(b_oe);
+      if (valid && half == 0) {
+        if (direct) {
+          if (p.lse) p.lse[(int64_t)tok * p.hq + h] = l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        } else {
+          s.part_ml[(int64_t)sg * kDcRows + r] = make_float2(m_used, l);
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Merge the pieces of every sequence that was split: block (row r, sequence b).
+template <typename T>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const AttnParams p, const DecodeSched s) {
+  const int r = blockIdx.x, b = blockIdx.y;
+  const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
+  if (r >= sq * p.hq) return;
+  const int cnt = s.seg_cnt[b];
+  if (cnt == 1) return;  // stored directly by the decode kernel
+  const int tok = q0 + r / p.hq, h = r % p.hq;
+  T *orow = reinterpret_cast<T *>(p.o) + (int64_t)tok * p.o_rs + (int64_t)h * p.o_hs;
+  const int base = s.seg_base[b];
+  float M = -INFINITY;
+  for (int i = 0; i < cnt; ++i) M = fmaxf(M, s.part_ml[(int64_t)(base + i) * kDcRows + r].x);
+  float L = 0.f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (M != -INFINITY) {
+    for (int i = 0; i < cnt; ++i) {
+      const float2 ml = s.part_ml[(int64_t)(base + i) * kDcRows + r];
+      const float w = ex2(ml.x - M);  // 0 for a piece that saw no visible key
+      L += w * ml.y;
+      const float4 a = reinterpret_cast<const float4 *>(s.part_acc + ((int64_t)(base + i) * kDcRows + r) * kDcDv)[threadIdx.x];
+      acc[0] = fmaf(w, a.x, acc[0]);
+      acc[1] = fmaf(w, a.y, acc[1]);
+      acc[2] = fmaf(w, a.z, acc[2]);
+      acc[3] = fmaf(w, a.w, acc[3]);
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const int d = threadIdx.x * 4;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) orow[d + e] = from_f32<T>(acc[e] * inv);
+  if (threadIdx.x == 0 && p.lse)
+    p.lse[(int64_t)tok * p.hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
+}
+
+}  // namespace mxfa

@@ -5,6 +5,7 @@
 // the caller's stream.  It never allocates device memory and never
 // synchronises, except in strict-validation mode and in
 // mxfa_read_device_status, which are documented to.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -25,6 +26,7 @@
 #include "simt.cuh"
 #include "prefill_tc.cuh"
 #include "sched.cuh"
+#include "decode_tc.cuh"
 
 using namespace mxfa;
 
@@ -130,6 +132,25 @@ mxfa_status_t make_map(CUtensorMap *map, const void *base, mxfa_dtype_t dt, int 
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MXFA_ERR_INVALID_ARG, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MXFA_OK;
+}
+
+// 2-D map over [rows][cols] (16-bit elements, row stride in elements), box =
+// 64 rows x 64 columns, 128-byte swizzle; rows past `rows` read as zero.
+mxfa_status_t make_map_2d(CUtensorMap *map, const void *base, mxfa_dtype_t dt, int cols, int64_t rows,
+                          int64_t row_stride) {
+  EncodeTiledFn enc;
+  mxfa_status_t st = get_encoder(&enc);
+  if (st != MXFA_OK) return st;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dt == MXFA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                   const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MXFA_ERR_INVALID_ARG, "cuTensorMapEncodeTiled (2-D) failed (%d)", (int)r);
   return MXFA_OK;
 }
 
@@ -261,6 +282,69 @@ mxfa_status_t prefill(AttnParams &p, mxfa_dtype_t dt, int D, bool varlen, int64_
   return bf ? launch_tc<64, true>(p, mq, mk, mv, st) : launch_tc<64, false>(p, mq, mk, mv, st);
 }
 
+// Workspace layout of the tensor-core MLA decode.
+struct DecodeWs {
+  size_t n_tiles, tile_pre, seg_base, seg_cnt, segs, part_ml, part_acc, total;
+  int max_segs;
+};
+DecodeWs decode_ws(int batch, int max_kv_len, int num_splits) {
+  DecodeWs w;
+  const int tiles = (max_kv_len + kDcKeys - 1) / kDcKeys;
+  w.max_segs = num_splits > 0 ? batch * std::max(1, std::min(num_splits, tiles)) : batch + kDcMaxGrid;
+  w.n_tiles = sizeof(WsHeader);
+  w.tile_pre = w.n_tiles + align256(sizeof(int) * (size_t)batch);
+  w.seg_base = w.tile_pre + align256(sizeof(int) * (size_t)(batch + 1));
+  w.seg_cnt = w.seg_base + align256(sizeof(int) * (size_t)(batch + 1));
+  w.segs = w.seg_cnt + align256(sizeof(int) * (size_t)batch);
+  w.part_ml = w.segs + align256(sizeof(int4) * (size_t)w.max_segs);
+  w.part_acc = w.part_ml + align256(sizeof(float2) * (size_t)w.max_segs * kDcRows);
+  w.total = w.part_acc + align256(sizeof(float) * (size_t)w.max_segs * kDcRows * kDcDv);
+  return w;
+}
+
+bool decode_tc_eligible(mxfa_dtype_t dt, int Hq, int Hkv, int Dqk, int Dv, int max_q_len, const void *k,
+                        const void *v, int64_t k_rs, int64_t v_rs) {
+  return dt != MXFA_F32 && Dqk == kDcDqk && Dv == kDcDv && Hkv == 1 && k == v && k_rs == v_rs &&
+         (int64_t)max_q_len * Hq <= kDcRows;
+}
+
+mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int total_kv, int num_splits, void *ws,
+                               cudaStream_t st) {
+  int sms = 0;
+  MXFA_TRY(sm_count(&sms));
+  const DecodeWs w = decode_ws(p.batch, p.max_sk, num_splits);
+  char *base = static_cast<char *>(ws);
+  DecodeSched s;
+  s.n_tiles = reinterpret_cast<int *>(base + w.n_tiles);
+  s.tile_pre = reinterpret_cast<int *>(base + w.tile_pre);
+  s.seg_base = reinterpret_cast<int *>(base + w.seg_base);
+  s.seg_cnt = reinterpret_cast<int *>(base + w.seg_cnt);
+  s.segs = reinterpret_cast<int4 *>(base + w.segs);
+  s.part_ml = reinterpret_cast<float2 *>(base + w.part_ml);
+  s.part_acc = reinterpret_cast<float *>(base + w.part_acc);
+  s.max_segs = w.max_segs;
+  s.num_splits = num_splits;
+  s.grid = std::min(sms, kDcMaxGrid);
+  CUtensorMap mq, mkv;
+  MXFA_TRY(make_map_2d(&mq, p.q, dt, kDcDqk, (int64_t)total_q * p.hq, kDcDqk));
+  MXFA_TRY(make_map_2d(&mkv, p.k, dt, kDcDqk, total_kv, p.k_rs));
+  decode_prep_kernel<<<1, 1024, 0, st>>>(p, s);
+  MXFA_CUDA(cudaGetLastError());
+  if (dt == MXFA_BF16) {
+    MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(attn_decode_tc_kernel<true>), kDcSmemBytes));
+    attn_decode_tc_kernel<true><<<s.grid, kDcThreads, kDcSmemBytes, st>>>(p, s, mq, mkv);
+    MXFA_CUDA(cudaGetLastError());
+    decode_combine_kernel<__nv_bfloat16><<<dim3(kDcRows, p.batch), 128, 0, st>>>(p, s);
+  } else {
+    MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(attn_decode_tc_kernel<false>), kDcSmemBytes));
+    attn_decode_tc_kernel<false><<<s.grid, kDcThreads, kDcSmemBytes, st>>>(p, s, mq, mkv);
+    MXFA_CUDA(cudaGetLastError());
+    decode_combine_kernel<__half><<<dim3(kDcRows, p.batch), 128, 0, st>>>(p, s);
+  }
+  MXFA_CUDA(cudaGetLastError());
+  return MXFA_OK;
+}
+
 mxfa_status_t check_heads(int Hq, int Hkv) {
   if (Hq <= 0 || Hkv <= 0) return fail(MXFA_ERR_INVALID_ARG, "head counts must be positive (Hq=%d, Hkv=%d)", Hq, Hkv);
   if (Hq % Hkv) return fail(MXFA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
@@ -388,8 +472,11 @@ mxfa_status_t mxfa_attn_varlen_fwd(const void *q, const void *k, const void *v, 
   return prefill(p, dtype, D, true, total_q, total_k, workspace, st);
 }
 
-size_t mxfa_attn_decode_splitkv_workspace_size(int, int, int, int, int, int, mxfa_dtype_t) {
-  return sizeof(WsHeader);
+size_t mxfa_attn_decode_splitkv_workspace_size(int batch, int max_q_len, int Hq, int Dv, int max_kv_len,
+                                               int num_splits, mxfa_dtype_t dtype) {
+  if (dtype == MXFA_F32 || Dv != kDcDv || batch <= 0 || (int64_t)max_q_len * Hq > kDcRows || num_splits < 0)
+    return sizeof(WsHeader);
+  return decode_ws(batch, max_kv_len, num_splits).total;
 }
 
 mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -440,6 +527,8 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
   p.causal = causal ? 1 : 0;
   p.hdr = static_cast<WsHeader *>(workspace);
   p.pairs = nullptr;
+  if (decode_tc_eligible(dtype, Hq, Hkv, Dqk, Dv, max_q_len, k, v, k_row_stride, v_row_stride) && total_kv > 0)
+    return launch_decode_tc(p, dtype, total_q, total_kv, num_splits, workspace, st);
   return launch_simt_any(dtype, p, max_q_len, st);
 }
 

@@ -183,6 +183,42 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 #undef MXFA_R8
 #undef MXFA_W8
 
+
+// 16-lane access ("16x32bx2", the two halves adjacent): threads 0-15 read
+// lanes base..base+15 at columns [c, c+32), threads 16-31 read the same lanes
+// at columns [c+32, c+64).  Touches only 16 lanes of the warp's sub-partition.
+#define MXFA_R8(i) "=r"(r[i + 0]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), \
+                   "=r"(r[i + 6]), "=r"(r[i + 7])
+#define MXFA_W8(i) "r"(r[i + 0]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), \
+                   "r"(r[i + 6]), "r"(r[i + 7])
+__device__ __forceinline__ void tmem_ld_half32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : MXFA_R8(0), MXFA_R8(8), MXFA_R8(16), MXFA_R8(24)
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_half32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 32, {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      MXFA_W8(0), MXFA_W8(8), MXFA_W8(16), MXFA_W8(24)
+      : "memory");
+}
+#undef MXFA_R8
+#undef MXFA_W8
+
+// 2-D tiled bulk tensor load global -> shared::cta, completion on `bar`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- math
 // 2^x on the multi-function unit (ex2.approx: 2 ulp; 2^-inf = +0).
 __device__ __forceinline__ float ex2(float x) {
