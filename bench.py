@@ -237,6 +237,8 @@ def main():
     ap.add_argument("--impl", default="mxfa", choices=["mxfa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-batch", type=int, default=128,
+                    help="sequences of the MLA decode workload (128 = the full workload; smaller for captures)")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="time one workload only (used for profiling captures)")
     args = ap.parse_args()
@@ -318,7 +320,8 @@ def main():
     # ---------------- decode (secondary measurement)
     decode = None
     if not args.no_decode and args.only != "prefill":
-        pdc = workloads.cfg_mla_decode()
+        pdc = (workloads.cfg_mla_decode() if args.decode_batch == 128 else
+               workloads.mla_decode(3, args.decode_batch, 4, 8192, name=f"mla_decode_b{args.decode_batch}_q4_h16_kv8192_bf16"))
         dd = to_dev(pdc, dev)
         od = torch.empty((pdc.total_q, pdc.hq, pdc.dv), dtype=torch.bfloat16, device=dev)
         ld = torch.empty((pdc.total_q, pdc.hq), dtype=torch.float32, device=dev)

@@ -7,13 +7,19 @@
 // sequence are flattened r = q*Hq + h and form the M = 64 side of every MMA.
 //
 // The KV cache is streamed exactly once: 64-key tiles arrive by TMA as nine
-// 8 KB column chunks (64 keys x 64 columns, 128B swizzle) into an 18-slot
-// ring (two tiles).  Each tile is used twice while resident:
-//     S   = Q K^T   tcgen05.mma M=64 N=64, 9 chunks x 4 K-steps, A = Q (smem)
+// 8 KB column chunks (64 keys x 64 columns, 128B swizzle) into a 27-slot
+// ring (three tiles, so two tiles are in flight while one is computed).
+// Each tile is used twice while resident:
+//     S   = Q K^T   tcgen05.mma M=64 N=64, 36 K-steps, A = Q (TMEM), B = K;
+//                   the K-steps go round-robin into three accumulators
+//                   (chunk c into chain c % 3) so consecutive MMAs do not
+//                   wait on each other; softmax adds the three
 //     O  += P V     tcgen05.mma M=64 N=256 (x2), A = P (smem), B = chunks 0-7
-// S lives in TMEM lanes 16-31 of each sub-partition (double-buffered), O in
-// lanes 0-15 (all 512 columns): the two M=64 accumulators interleave in
-// TMEM.  A softmax warpgroup (128 threads) gives each query row two threads,
+// TMEM: O in lanes 0-15 of each sub-partition (all 512 columns); in lanes
+// 16-31 the three S chains (columns 0-191) and Q (columns 192-479, two bf16
+// per column), so the shared-memory budget goes to the KV ring.  S has one
+// buffer: softmax signals as soon as it has read S(j), and S(j+1) is issued
+// before P.V(j).  A softmax warpgroup (128 threads) gives each query row two threads,
 // one per 32-key half of the tile (16-lane TMEM accesses), with the online
 // softmax of the prefill kernel (exp2 domain, rescale of O only when the
 // row max grows by more than 2^8).
@@ -40,10 +46,12 @@ constexpr int kDcKeys = 64;       // keys per tile
 constexpr int kDcDqk = 576, kDcDv = 512;
 constexpr int kDcChunks = kDcDqk / 64;  // 9 column chunks per KV tile
 constexpr int kDcChunkBytes = kDcKeys * 128;
-constexpr int kDcSlots = 2 * kDcChunks;
+constexpr int kDcRingTiles = 3;
+constexpr int kDcSlots = kDcRingTiles * kDcChunks;
+constexpr int kDcQCol = 192;  // first TMEM column of Q (lanes 16-31); S chains use 0-191
 constexpr int kDcThreads = 256;
 constexpr int kDcCtrlBytes = 2048;
-constexpr int kDcSmemBytes = kDcCtrlBytes + (kDcChunks + kDcSlots) * kDcChunkBytes + kDcRows * 128;
+constexpr int kDcSmemBytes = kDcCtrlBytes + kDcSlots * kDcChunkBytes + kDcRows * 128;
 static_assert(kDcSmemBytes <= 232448, "shared memory budget");
 constexpr int kDcMaxGrid = 256;
 
@@ -61,17 +69,17 @@ struct DecodeSched {
 };
 
 struct DecodeCtrl {
-  uint64_t q_full, q_empty;
-  uint64_t slot_full[kDcSlots], slot_empty[kDcSlots];
-  uint64_t s_full[2], p_full, o_done, o_empty;
+  uint64_t q_ready;
+  uint64_t tile_full[kDcRingTiles], tile_empty[kDcRingTiles];
+  uint64_t s_full, s_free, p_full, o_done, o_empty;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
 
 enum : uint32_t {
-  kDSiteQEmpty = 0x301, kDSiteSlotEmpty, kDSiteQFull, kDSiteSlotFull, kDSitePFull, kDSiteOEmpty, kDSiteSFull,
-  kDSiteODone
+  kDSiteSlotEmpty = 0x301, kDSiteQReady, kDSiteSlotFull, kDSitePFull, kDSiteOEmpty, kDSiteSFull,
+  kDSiteODone, kDSiteSFree
 };
 
 __device__ __forceinline__ int dc_range_start(int c, int T, int G) { return (int)(((int64_t)c * T) / G); }
@@ -183,28 +191,26 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
   extern __shared__ uint8_t smem_raw[];
   DecodeCtrl *ctrl = reinterpret_cast<DecodeCtrl *>(smem_raw);
   const uint32_t tiles_u32 = (smem_u32(smem_raw) + 1024u + 1023u) & ~1023u;
-  const uint32_t q_u32 = tiles_u32;                                  // 9 chunks of Q
-  const uint32_t ring_u32 = q_u32 + kDcChunks * kDcChunkBytes;       // 18 KV chunk slots
+  const uint32_t ring_u32 = tiles_u32;                               // 3 tiles x 9 KV chunks
   const uint32_t p_u32 = ring_u32 + kDcSlots * kDcChunkBytes;        // P: 64 rows x 128 B
   uint8_t *p_gen = smem_raw + (p_u32 - smem_u32(smem_raw));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int *abort_flag = &ctrl->abort;
   WsHeader *hdr = p.hdr;
-  auto b_sf = [&](int x) { return smem_u32(&ctrl->slot_full[x]); };
-  auto b_se = [&](int x) { return smem_u32(&ctrl->slot_empty[x]); };
-  const uint32_t b_qf = smem_u32(&ctrl->q_full), b_qe = smem_u32(&ctrl->q_empty);
+  auto b_tf = [&](int x) { return smem_u32(&ctrl->tile_full[x]); };
+  auto b_te = [&](int x) { return smem_u32(&ctrl->tile_empty[x]); };
+  const uint32_t b_qr = smem_u32(&ctrl->q_ready), b_sf = smem_u32(&ctrl->s_full), b_sx = smem_u32(&ctrl->s_free);
   const uint32_t b_pf = smem_u32(&ctrl->p_full), b_od = smem_u32(&ctrl->o_done), b_oe = smem_u32(&ctrl->o_empty);
 
   if (threadIdx.x == 0) {
-    mbar_init(b_qf, 1);
-    mbar_init(b_qe, 1);
-    for (int x = 0; x < kDcSlots; ++x) {
-      mbar_init(b_sf(x), 1);
-      mbar_init(b_se(x), 1);
+    mbar_init(b_qr, 128);
+    for (int x = 0; x < kDcRingTiles; ++x) {
+      mbar_init(b_tf(x), 1);
+      mbar_init(b_te(x), 1);
     }
-    mbar_init(smem_u32(&ctrl->s_full[0]), 1);
-    mbar_init(smem_u32(&ctrl->s_full[1]), 1);
+    mbar_init(b_sf, 1);
+    mbar_init(b_sx, 128);
     mbar_init(b_pf, 128);
     mbar_init(b_od, 1);
     mbar_init(b_oe, 128);
@@ -212,10 +218,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     ctrl->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_kv);
-  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_kv);
   if (warp == 1) {
     tmem_alloc(smem_u32(&ctrl->tmem_base), 512);
     tmem_relinquish();
@@ -234,36 +237,35 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t ring = 0, q_issued = 0;
+      uint32_t tc = 0;  // tiles issued by this CTA
       bool ok = true;
       for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
         const int4 sd = s.segs[sg];
-        const int q0 = p.cu_q[sd.x], k0 = p.cu_k[sd.x];
-        if (q_issued > 0 && !wait_bar(b_qe, (q_issued - 1) & 1, abort_flag, hdr, kDSiteQEmpty)) break;
-        mbar_arrive_expect_tx(b_qf, kDcChunks * kDcChunkBytes);
-        for (int c = 0; c < kDcChunks; ++c)
-          tma_load_2d(q_u32 + c * kDcChunkBytes, &tm_q, b_qf, c * 64, q0 * p.hq);
-        ++q_issued;
-        for (int j = sd.y; ok && j < sd.z; ++j) {
-          for (int c = 0; c < kDcChunks; ++c, ++ring) {
-            const int x = ring % kDcSlots;
-            if (!wait_bar(b_se(x), ((ring / kDcSlots) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(b_sf(x), kDcChunkBytes);
-            tma_load_2d(ring_u32 + x * kDcChunkBytes, &tm_kv, b_sf(x), c * 64, k0 + j * kDcKeys);
+        const int k0 = p.cu_k[sd.x];
+        if (sg + 1 < seg_hi) {  // the next piece's query rows, into L2
+          const int bn = s.segs[sg + 1].x;
+          const int64_t q0n = p.cu_q[bn], rn = (p.cu_q[bn + 1] - q0n) * p.hq;
+          if (rn > 0)
+            tma_prefetch_bytes(reinterpret_cast<const uint16_t *>(p.q) + q0n * p.hq * kDcDqk,
+                               (uint32_t)(rn * kDcDqk * 2));
+        }
+        for (int j = sd.y; ok && j < sd.z; ++j, ++tc) {
+          const int x = tc % kDcRingTiles;
+          if (!wait_bar(b_te(x), ((tc / kDcRingTiles) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty)) {
+            ok = false;
+            break;
           }
+          mbar_arrive_expect_tx(b_tf(x), kDcChunks * kDcChunkBytes);
+          for (int c = 0; c < kDcChunks; ++c)
+            tma_load_2d(ring_u32 + (x * kDcChunks + c) * kDcChunkBytes, &tm_kv, b_tf(x), c * 64, k0 + j * kDcKeys);
         }
       }
+      // Teardown: every tile load this thread issued must have landed.
       const uint64_t t0 = global_ns();
-      if (q_issued > 0)
-        while (!mbar_test(b_qf, (q_issued - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
-        }
-      for (int x = 0; x < kDcSlots; ++x) {
-        const uint32_t uses = ring / kDcSlots + ((uint32_t)x < ring % kDcSlots ? 1u : 0u);
+      for (int x = 0; x < kDcRingTiles; ++x) {
+        const uint32_t uses = tc / kDcRingTiles + ((uint32_t)x < tc % kDcRingTiles ? 1u : 0u);
         if (uses == 0) continue;
-        while (!mbar_test(b_sf(x), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        while (!mbar_test(b_tf(x), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
         }
       }
     }
@@ -272,41 +274,38 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc_f16(BF16, kDcRows, kDcKeys, false, false);
       constexpr uint32_t idesc_o = make_idesc_f16(BF16, kDcRows, 256, false, true);
-      const uint32_t s_tmem = tmem + (16u << 16);  // S: lanes 16-31 of each sub-partition
-      uint32_t ring = 0, g = 0, o_uses = 0;
+      const uint32_t s_tmem = tmem + (16u << 16);  // S chains and Q: lanes 16-31 of each sub-partition
+      uint32_t tc = 0, g = 0, o_uses = 0;
       bool ok = true;
-      // S(tile) into buffer buf; the tile's chunks start at ring slot `first`.
-      auto issue_s = [&](uint32_t buf, uint32_t first) -> bool {
-        for (int c = 0; c < kDcChunks; ++c) {
-          const uint32_t x = (first + c) % kDcSlots;
-          if (!wait_bar(b_sf(x), ((first + c) / kDcSlots) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
-          tc_fence_after();
+      // S of tile counter `t` into the three chains (chunk c accumulates into chain c % 3).
+      auto issue_s = [&](uint32_t t) -> bool {
+        const int x = t % kDcRingTiles;
+        if (!wait_bar(b_tf(x), (t / kDcRingTiles) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
+        tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(s_tmem + buf * kDcKeys, make_sdesc_sw128(q_u32 + c * kDcChunkBytes + kk * 32, 16, 1024),
-                   make_sdesc_sw128(ring_u32 + x * kDcChunkBytes + kk * 32, 16, 1024), idesc_s,
-                   (c > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(smem_u32(&ctrl->s_full[buf]));
-        mma_commit(b_se((first + kDcChunks - 1) % kDcSlots));  // the rope chunk is only read by S
+        for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+          for (int c = 0; c < kDcChunks; ++c)
+            mma_ts(s_tmem + (c % 3) * kDcKeys, s_tmem + kDcQCol + (c * 4 + kk) * 8,
+                   make_sdesc_sw128(ring_u32 + (x * kDcChunks + c) * kDcChunkBytes + kk * 32, 16, 1024), idesc_s,
+                   (c >= 3 || kk > 0) ? 1u : 0u);
+        mma_commit(b_sf);
         return true;
       };
       for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
         const int4 sd = s.segs[sg];
         const int n = sd.z - sd.y;
-        if (!wait_bar(b_qf, (sg - seg_lo) & 1, abort_flag, hdr, kDSiteQFull)) break;
+        if (!wait_bar(b_qr, (sg - seg_lo) & 1, abort_flag, hdr, kDSiteQReady)) break;
         tc_fence_after();
-        if (!issue_s(g & 1, ring)) break;
-        if (n == 1) mma_commit(b_qe);
-        for (int jj = 0; jj < n; ++jj, ++g) {
-          const uint32_t first = ring;
-          ring += kDcChunks;
+        if (g > 0 && !wait_bar(b_sx, (g - 1) & 1, abort_flag, hdr, kDSiteSFree)) break;
+        if (!issue_s(tc)) break;
+        for (int jj = 0; jj < n; ++jj, ++g, ++tc) {
           if (jj + 1 < n) {
-            if (!issue_s((g + 1) & 1, ring)) {
+            // the single S buffer is free once softmax has read S(g)
+            if (!wait_bar(b_sx, g & 1, abort_flag, hdr, kDSiteSFree) || !issue_s(tc + 1)) {
               ok = false;
               break;
             }
-            if (jj + 2 == n) mma_commit(b_qe);
           }
           if (!wait_bar(b_pf, g & 1, abort_flag, hdr, kDSitePFull)) {
             ok = false;
@@ -317,17 +316,16 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
             break;
           }
           tc_fence_after();
+          const uint32_t vbase = ring_u32 + (tc % kDcRingTiles) * kDcChunks * kDcChunkBytes;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const uint32_t vfirst = (first + half * 4) % kDcSlots;  // chunks 4*half..4*half+3 are consecutive
+          for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
+            for (int half = 0; half < 2; ++half)
               mma_ss(tmem + half * 256, make_sdesc_sw128(p_u32 + kk * 32, 16, 1024),
-                     make_sdesc_sw128(ring_u32 + vfirst * kDcChunkBytes + kk * 16 * 128, kDcChunkBytes, 1024),
+                     make_sdesc_sw128(vbase + half * 4 * kDcChunkBytes + kk * 16 * 128, kDcChunkBytes, 1024),
                      idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
-          }
           mma_commit(b_od);
-          for (int c = 0; c < kDcChunks - 1; ++c) mma_commit(b_se((first + c) % kDcSlots));
+          mma_commit(b_te(tc % kDcRingTiles));
         }
         ++o_uses;
       }
@@ -344,8 +342,45 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     const uint32_t s_row = tmem + ((uint32_t)(sub * 32 + 16) << 16);
     const float c = p.scale_log2;
     const bool neg = c < 0.f;
+    // Q rows of piece sg into TMEM (lanes 16-31, columns kDcQCol..): this
+    // thread writes half `half` of row r; all global loads are issued first.
+    auto load_q = [&](int sg) {
+      const int bq = s.segs[sg].x;
+      const int q0 = p.cu_q[bq], rows = (p.cu_q[bq + 1] - q0) * p.hq;
+      const uint4 *src = reinterpret_cast<const uint4 *>(
+          reinterpret_cast<const uint16_t *>(p.q) + ((int64_t)q0 * p.hq + r) * kDcDqk);
+      const bool vq = r < rows;
+#pragma unroll
+      for (int k2 = 0; k2 < 2; ++k2) {
+        uint4 w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = vq ? src[(k2 * 2 + i / 8) * 16 + half * 8 + (i & 7)] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int k1 = 0; k1 < 2; ++k1) {
+          uint32_t v[32];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint4 u = w[k1 * 8 + i];
+            v[4 * i] = u.x; v[4 * i + 1] = u.y; v[4 * i + 2] = u.z; v[4 * i + 3] = u.w;
+          }
+          tmem_st_half32(s_row + kDcQCol + (k2 * 2 + k1) * 64, v);
+        }
+      }
+      uint32_t v[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 u = vq ? src[64 + half * 4 + i] : make_uint4(0, 0, 0, 0);
+        v[4 * i] = u.x; v[4 * i + 1] = u.y; v[4 * i + 2] = u.z; v[4 * i + 3] = u.w;
+      }
+      tmem_st_half16(s_row + kDcQCol + 256, v);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(b_qr);
+    };
     uint32_t g = 0;
     bool ok = true;
+    if (seg_lo < seg_hi) load_q(seg_lo);
     for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
       const int4 sd = s.segs[sg];
       const int b = sd.x;
@@ -355,15 +390,23 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       const int nv = valid ? visible_keys(r / p.hq, sq, sk, p.causal) : 0;
       float m_used = -INFINITY, l = 0.f;
       for (int j = sd.y; j < sd.z; ++j, ++g) {
-        const bool got = wait_bar(smem_u32(&ctrl->s_full[g & 1]), (g >> 1) & 1, abort_flag, hdr, kDSiteSFull);
+        const bool got = wait_bar(b_sf, g & 1, abort_flag, hdr, kDSiteSFull);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t sv[32];
-        tmem_ld_half32(s_row + (g & 1) * kDcKeys, sv);
+        uint32_t sv[32], sb[32];
+        tmem_ld_half32(s_row + 0 * kDcKeys, sv);
+        tmem_ld_half32(s_row + 1 * kDcKeys, sb);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sv[e] = __float_as_uint(__uint_as_float(sv[e]) + __uint_as_float(sb[e]));
+        tmem_ld_half32(s_row + 2 * kDcKeys, sb);
+        tc_fence_before();
+        mbar_arrive(b_sx);  // S may be overwritten now
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sv[e] = __float_as_uint(__uint_as_float(sv[e]) + __uint_as_float(sb[e]));
         const int lim = nv - j * kDcKeys - half * 32;  // keys [0, lim) of this half are visible
         float ext = -INFINITY;
 #pragma unroll
@@ -429,6 +472,8 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         mbar_arrive(b_pf);
       }
       if (!ok) break;
+      // Every S of this piece has been read, so Q of the next piece may go in.
+      if (sg + 1 < seg_hi) load_q(sg + 1);
       // ---------------- epilogue of this piece
       l += __shfl_xor_sync(0xffffffffu, l, 16);
       if (sd.z > sd.y) {

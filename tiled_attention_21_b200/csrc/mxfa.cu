@@ -96,6 +96,24 @@ mxfa_status_t ensure_smem(const void *kernel, size_t bytes) {
   return MXFA_OK;
 }
 
+// A kernel that moves registers between warpgroups (setmaxnreg) is only
+// safe with the per-thread register count its split was computed for.
+std::set<const void *> g_regs_ok;
+mxfa_status_t check_launch_regs(const void *kernel, int expected) {
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (g_regs_ok.count(kernel)) return MXFA_OK;
+  }
+  cudaFuncAttributes a;
+  MXFA_CUDA(cudaFuncGetAttributes(&a, kernel));
+  if (a.numRegs != expected)
+    return fail(MXFA_ERR_UNSUPPORTED, "kernel built with %d registers per thread, its register split needs %d",
+                a.numRegs, expected);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  g_regs_ok.insert(kernel);
+  return MXFA_OK;
+}
+
 // ---------------------------------------------------------------- TMA descriptors
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -236,6 +254,7 @@ mxfa_status_t launch_tc(const AttnParams &p, const CUtensorMap &mq, const CUtens
   int sms = 0;
   MXFA_TRY(sm_count(&sms));
   auto k = attn_fwd_tc_kernel<D, BF16>;
+  MXFA_TRY(check_launch_regs(reinterpret_cast<const void *>(k), kTcLaunchRegs));
   MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(k), PrefillCfg<D>::kSmemBytes));
   k<<<sms, kTcThreads, PrefillCfg<D>::kSmemBytes, st>>>(p, mq, mk, mv);
   MXFA_CUDA(cudaGetLastError());

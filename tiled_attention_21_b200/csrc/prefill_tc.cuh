@@ -18,14 +18,17 @@
 // more than 2^8.  Until then O and l keep the stale maximum as their common
 // base, which leaves O = acc / l and LSE = base + log2(l) exact.
 //
-// Roles (384 threads):
+// Roles (384 threads, three warpgroups):
 //   warp 0      TMA producer: Q tiles once per unit, then K_j, V_j into a
 //               ring of shared-memory slots (128B-swizzled boxes of 64 cols)
 //   warp 1      TMEM allocator and single-thread MMA issuer; it alternates
 //               the two query tiles (PV_0(j), S_0(j+1), PV_1(j), S_1(j+1))
 //               so one tile's softmax overlaps the other tile's MMAs
-//   warps 4-7   softmax + epilogue of query tile 0 (TMEM lanes 0..127)
+//   warps 4-7   softmax + epilogue of query tile 0 (warp w reads TMEM lanes
+//               32*(w%4) .. 32*(w%4)+31, so the four warps cover rows 0..127)
 //   warps 8-11  softmax + epilogue of query tile 1
+// The first warpgroup gives registers to the other two (setmaxnreg) so a
+// softmax thread keeps its whole 128-column score row in registers.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
 //
 // Every wait is bounded (see wait_bar); a wait that runs out records
@@ -37,6 +40,7 @@
 #include <type_traits>
 
 #include "ptx.cuh"
+#include "exp2_poly.cuh"
 
 namespace mxfa {
 
@@ -44,6 +48,13 @@ constexpr int kTcBlockM = 128;  // rows per query tile
 constexpr int kTcBlockN = 128;  // keys per KV tile
 constexpr int kTcUnitRows = 2 * kTcBlockM;
 constexpr int kTcThreads = 384;
+// Register split (setmaxnreg): launched at kTcLaunchRegs per thread, the
+// producer/MMA warpgroup drops to kTcRegsIo and the two softmax warpgroups
+// rise to kTcRegsSoftmax; 128*kTcRegsIo + 256*kTcRegsSoftmax must not exceed
+// 384*kTcLaunchRegs (the host refuses to launch a build whose register count
+// differs from kTcLaunchRegs).
+constexpr int kTcLaunchRegs = 168, kTcRegsIo = 72, kTcRegsSoftmax = 216;
+static_assert(128 * kTcRegsIo + 256 * kTcRegsSoftmax <= kTcThreads * kTcLaunchRegs, "register split");
 constexpr int kTcMaxSlots = 10;
 
 template <int D>
@@ -122,6 +133,90 @@ __device__ __forceinline__ int n_units_of(const AttnParams &p) {
   return (int)(*reinterpret_cast<volatile uint32_t *>(&p.hdr->n_units)) * p.hq;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t pk2(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Row maximum of the 128 scores of a tile (keys >= lim excluded when MASKED),
+// four independent chains of three-input maxima.
+template <bool MASKED>
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[128], int lim) {
+  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int q = 0; q < 128; q += 2) {
+    float a = __uint_as_float(sr[q]), b = __uint_as_float(sr[q + 1]);
+    if (MASKED) {
+      a = q < lim ? a : -INFINITY;
+      b = q + 1 < lim ? b : -INFINITY;
+    }
+    m4[(q >> 1) & 3] = fmax3(m4[(q >> 1) & 3], a, b);
+  }
+  return fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+}
+
+// P = 2^(c*s - base) for the 128 scores, written into TMEM over S as packed
+// 16-bit pairs; returns the fp32 row sum.  Score pairs go through the packed
+// fp32x2 FMA; three of every eight pairs are exponentiated by the FMA-pipe
+// polynomial, the rest by the multi-function unit.
+template <bool MASKED, bool BF16>
+__device__ __forceinline__ float exp_store(const uint32_t (&sr)[128], int lim, float c, float base, uint32_t taddr) {
+  const uint64_t c2 = pk2(__float_as_uint(c), __float_as_uint(c));
+  const uint64_t nb2 = pk2(__float_as_uint(-base), __float_as_uint(-base));
+  uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int c0 = q * 32 + 2 * e;
+      const uint64_t x = ffma2(pk2(sr[c0], sr[c0 + 1]), c2, nb2);
+      float p0, p1;
+      if ((e & 7) >= 5) {
+        upk2(exp2_poly2(x), p0, p1);
+      } else {
+        float x0, x1;
+        upk2(x, x0, x1);
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+      }
+      if (MASKED) {
+        p0 = c0 < lim ? p0 : 0.f;
+        p1 = c0 + 1 < lim ? p1 : 0.f;
+      }
+      acc[e & 3] = fadd2(acc[e & 3], pk2(__float_as_uint(p0), __float_as_uint(p1)));
+      pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+    }
+    tmem_st16(taddr + q * 16, pk);
+  }
+  tmem_wait_st();
+  acc[0] = fadd2(acc[0], acc[1]);
+  acc[2] = fadd2(acc[2], acc[3]);
+  acc[0] = fadd2(acc[0], acc[2]);
+  float lo, hi;
+  upk2(acc[0], lo, hi);
+  return lo + hi;
+}
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tm_q,
@@ -176,6 +271,8 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
   const int n_units = n_units_of(p);
   const int grid = gridDim.x, cta = blockIdx.x;
 
+  if (warp < 4) {
+  regs_dec<kTcRegsIo>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -328,15 +425,17 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < kWaitBudgetNs) {
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_inc<kTcRegsSoftmax>();
     // ------------------------------------------------------------ softmax / epilogue
     const int t = (warp - 4) >> 2;
     const int sub = warp & 3;
     const int r = sub * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16);
     const uint32_t s_col = t * kTcBlockN, o_col = 2 * kTcBlockN + t * D;
-    const float c = p.scale_log2;
-    const bool neg = c < 0.f;
+    const bool neg = p.scale_log2 < 0.f;
+    const float cpos = neg ? -p.scale_log2 : p.scale_log2;
     const uint32_t b_s = smem_u32(&ctrl->s_full[t]), b_p = smem_u32(&ctrl->p_full[t]);
     const uint32_t b_od = smem_u32(&ctrl->o_done[t]), b_oe = smem_u32(&ctrl->o_empty[t]);
     uint32_t s_cnt = 0, pv_cnt = 0;
@@ -359,29 +458,15 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         ++s_cnt;
         tc_fence_after();
         uint32_t sr[128];
-        tmem_ld32(trow + s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(trow + s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld32(trow + s_col + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        tmem_ld32(trow + s_col + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-        const int lim = nv - j * kTcBlockN;  // keys [0, lim) of this tile are visible
-        const bool masked = lim < kTcBlockN;
-        float ext = -INFINITY;
-        if (!masked) {
-          if (!neg) {
+        tmem_ld128(trow + s_col, sr);
+        if (neg) {  // c*s = (-c)*(-s): fold a negative scale into the scores once
 #pragma unroll
-            for (int q = 0; q < 128; ++q) ext = fmaxf(ext, __uint_as_float(sr[q]));
-          } else {
-#pragma unroll
-            for (int q = 0; q < 128; ++q) ext = fmaxf(ext, -__uint_as_float(sr[q]));
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 128; ++q) {
-            const float x = neg ? -__uint_as_float(sr[q]) : __uint_as_float(sr[q]);
-            ext = (q < lim) ? fmaxf(ext, x) : ext;
-          }
+          for (int q = 0; q < 128; ++q) sr[q] ^= 0x80000000u;
         }
-        const float m_tile = (ext == -INFINITY) ? -INFINITY : (neg ? -ext : ext) * c;
+        const int lim = nv - j * kTcBlockN;  // keys [0, lim) of this tile are visible
+        const bool masked = __any_sync(0xffffffffu, lim < kTcBlockN);
+        const float ext = masked ? row_max<true>(sr, lim) : row_max<false>(sr, lim);
+        const float m_tile = (ext == -INFINITY) ? -INFINITY : ext * cpos;
         const float m_new = fmaxf(m_used, m_tile);
         float alpha = 1.f;
         bool need = false;
@@ -393,27 +478,9 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
           need = true;
         }
         const float base = (m_used == -INFINITY) ? 0.f : m_used;
-        float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c0 = q * 32 + 2 * e;
-            float p0 = ex2(fmaf(__uint_as_float(sr[c0]), c, -base));
-            float p1 = ex2(fmaf(__uint_as_float(sr[c0 + 1]), c, -base));
-            if (masked) {
-              p0 = c0 < lim ? p0 : 0.f;
-              p1 = c0 + 1 < lim ? p1 : 0.f;
-            }
-            rs0 += p0;
-            rs1 += p1;
-            pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
-          }
-          tmem_st16(trow + s_col + q * 16, pk);
-        }
-        tmem_wait_st();
-        l = l * alpha + (rs0 + rs1);
+        const float rsum = masked ? exp_store<true, BF16>(sr, lim, cpos, base, trow + s_col)
+                                  : exp_store<false, BF16>(sr, lim, cpos, base, trow + s_col);
+        l = l * alpha + rsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // PV_t(j-1) is the latest accumulation into O_t; it must be done.
           const bool got_o = wait_bar(b_od, (pv_cnt - 1) & 1, abort_flag, hdr, kSiteODone);
