@@ -25,9 +25,10 @@
 // row max grows by more than 2^8).
 //
 // Work split (d1): the KV tiles of all sequences form one sequence of T
-// tiles; CTA c of G owns tiles [c*T/G, (c+1)*T/G) (automatic split), or each
-// sequence is cut into k near-equal pieces (num_splits = k) and a piece
-// belongs to the CTA whose range holds its first tile.  A sequence covered by
+// tiles; CTA c of G owns the pieces whose first tile lies in
+// [c*T/G, (c+1)*T/G).  Pieces are whole sequences, or (when that would
+// leave the CTAs badly unbalanced) the sequences cut at those boundaries, or
+// with num_splits = k every sequence cut into k near-equal pieces.  A sequence covered by
 // one piece is normalised and stored directly; otherwise every piece writes
 // its unnormalised partial (acc, running max, running sum) and
 // decode_combine_kernel merges them with weights 2^(m_s - max_s m_s).
@@ -96,13 +97,23 @@ __device__ __forceinline__ int dc_lower_bound(const int4 *segs, int n, int x) {
 
 // ----------------------------------------------------------------------------
 // Schedule: one 1024-thread CTA.
+//   n_tiles[b]   = ceil(kv_len_b / 64) (0 when the sequence has no queries)
+//   tile_pre     = prefix of n_tiles (the global tile sequence)
+//   pieces       = num_splits > 0: min(k, n_b) near-equal pieces per sequence;
+//                  automatic: whole sequences, unless cutting the global tile
+//                  sequence at the CTA boundaries c*T/G shortens the longest
+//                  CTA by more than a fifth (splitting costs partial writes,
+//                  a combine pass and an extra Q load per piece).
 __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, DecodeSched s) {
   using Scan = cub::BlockScan<int, 1024>;
   __shared__ typename Scan::TempStorage tmp;
-  __shared__ int carry;
+  __shared__ int carry, max_n, split_mode;
+  __shared__ int cut[kDcMaxGrid + 1];  // x_c = c*T/G, c = 0..G
   const int tid = threadIdx.x, B = p.batch, G = s.grid;
-  // tiles per sequence and their prefix
-  if (tid == 0) carry = 0;
+  if (tid == 0) {
+    carry = 0;
+    max_n = 0;
+  }
   __syncthreads();
   for (int base = 0; base < B; base += 1024) {
     const int b = base + tid;
@@ -111,6 +122,7 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
       n = (p.cu_k[b + 1] - p.cu_k[b] + kDcKeys - 1) / kDcKeys;
       if (p.cu_q[b + 1] - p.cu_q[b] <= 0) n = 0;  // no queries: nothing to compute
       s.n_tiles[b] = n;
+      atomicMax(&max_n, n);
     }
     int incl, total;
     Scan(tmp).InclusiveSum(n, incl, total);
@@ -121,19 +133,36 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
   }
   if (tid == 0) s.tile_pre[0] = 0;
   const int T = carry;
+  for (int c = tid; c <= G; c += 1024) cut[c] = (int)(((int64_t)c * T) / G);
+  if (tid == 0) {
+    // longest CTA with whole sequences (they are dealt out by first tile) vs. the even cut
+    const int64_t whole = (int64_t)max_n * ((B + G - 1) / G);
+    const int64_t even = (T + G - 1) / G;
+    split_mode = (s.num_splits > 0) ? 1 : (5 * whole > 6 * even ? 2 : 0);  // 0 whole, 1 k pieces, 2 even cut
+  }
   __syncthreads();
-  // pieces per sequence
+  // first c with cut[c] > x (cut is non-decreasing)
+  auto upper = [&](int x) {
+    int lo = 0, hi = G + 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (cut[mid] <= x) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+  };
   auto pieces = [&](int b) -> int {
     const int n = s.n_tiles[b];
     if (n == 0) return 0;
-    if (s.num_splits > 0) return min(s.num_splits, n);
+    if (split_mode == 0) return 1;
+    if (split_mode == 1) return min(s.num_splits, n);
+    // distinct cut values strictly inside (P, P + n)
     const int P = s.tile_pre[b];
-    int cuts = 0;
-    for (int c = 1; c < G; ++c) {
-      const int x = dc_range_start(c, T, G);
-      // distinct boundaries strictly inside the sequence's tile range
-      cuts += (x > P && x < P + n && x != dc_range_start(c - 1, T, G)) ? 1 : 0;
-    }
+    int cuts = 0, prev = P;
+    for (int c = upper(P); c < G && cut[c] < P + n; ++c)
+      if (cut[c] != prev) {
+        ++cuts;
+        prev = cut[c];
+      }
     return 1 + cuts;
   };
   if (tid == 0) carry = 0;
@@ -152,12 +181,11 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
   const int n_segs = carry;
   if (tid == 0) s.seg_base[B] = n_segs;
   __syncthreads();
-  // the pieces themselves
   for (int b = tid; b < B; b += 1024) {
     const int n = s.n_tiles[b], P = s.tile_pre[b], k = s.seg_cnt[b];
     int idx = s.seg_base[b];
     if (k == 0) continue;
-    if (s.num_splits > 0) {
+    if (split_mode == 1) {
       for (int i = 0; i < k; ++i) {
         const int t0 = (int)(((int64_t)i * n) / k), t1 = (int)(((int64_t)(i + 1) * n) / k);
         if (idx < s.max_segs) s.segs[idx] = make_int4(b, t0, t1, P + t0);
@@ -165,12 +193,13 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
       }
     } else {
       int t0 = 0;
-      for (int c = 1; c <= G; ++c) {
-        const int x = c < G ? dc_range_start(c, T, G) : P + n;
-        if (x > P + t0 && x < P + n) {
-          if (idx < s.max_segs) s.segs[idx] = make_int4(b, t0, x - P, P + t0);
-          ++idx;
-          t0 = x - P;
+      if (split_mode == 2) {
+        for (int c = upper(P); c < G && cut[c] < P + n; ++c) {
+          if (cut[c] > P + t0) {
+            if (idx < s.max_segs) s.segs[idx] = make_int4(b, t0, cut[c] - P, P + t0);
+            ++idx;
+            t0 = cut[c] - P;
+          }
         }
       }
       if (idx < s.max_segs) s.segs[idx] = make_int4(b, t0, n, P + t0);
