@@ -18,17 +18,19 @@
 // more than 2^8.  Until then O and l keep the stale maximum as their common
 // base, which leaves O = acc / l and LSE = base + log2(l) exact.
 //
-// Roles (384 threads, three warpgroups):
+// Roles (640 threads, five warpgroups):
 //   warp 0      TMA producer: Q tiles once per unit, then K_j, V_j into a
 //               ring of shared-memory slots (128B-swizzled boxes of 64 cols)
 //   warp 1      TMEM allocator and single-thread MMA issuer; it alternates
 //               the two query tiles (PV_0(j), S_0(j+1), PV_1(j), S_1(j+1))
 //               so one tile's softmax overlaps the other tile's MMAs
-//   warps 4-7   softmax + epilogue of query tile 0 (warp w reads TMEM lanes
-//               32*(w%4) .. 32*(w%4)+31, so the four warps cover rows 0..127)
-//   warps 8-11  softmax + epilogue of query tile 1
-// The first warpgroup gives registers to the other two (setmaxnreg) so a
-// softmax thread keeps its whole 128-column score row in registers.
+//   warps 4-11  softmax + epilogue of query tile 0, warps 12-19 of tile 1.
+//               A query row has two threads in two warps of the same TMEM
+//               sub-partition (warp w reads lanes 32*(w%4)..+31): one takes
+//               key columns 0-63 and output columns 0..D/2-1, the other the
+//               upper halves; they swap partial row maxima through shared
+//               memory (a 64-thread named barrier per pair of warps).
+// The first warpgroup gives registers to the softmax warpgroups (setmaxnreg).
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
 //
 // Every wait is bounded (see wait_bar); a wait that runs out records
@@ -47,14 +49,15 @@ namespace mxfa {
 constexpr int kTcBlockM = 128;  // rows per query tile
 constexpr int kTcBlockN = 128;  // keys per KV tile
 constexpr int kTcUnitRows = 2 * kTcBlockM;
-constexpr int kTcThreads = 384;
+constexpr int kTcThreads = 640;
+constexpr int kTcSoftmaxThreads = 512;  // four warpgroups: (query tile, column half)
 // Register split (setmaxnreg): launched at kTcLaunchRegs per thread, the
-// producer/MMA warpgroup drops to kTcRegsIo and the two softmax warpgroups
-// rise to kTcRegsSoftmax; 128*kTcRegsIo + 256*kTcRegsSoftmax must not exceed
-// 384*kTcLaunchRegs (the host refuses to launch a build whose register count
+// producer/MMA warpgroup drops to kTcRegsIo and the four softmax warpgroups
+// rise to kTcRegsSoftmax; 128*kTcRegsIo + 512*kTcRegsSoftmax must not exceed
+// 640*kTcLaunchRegs (the host refuses to launch a build whose register count
 // differs from kTcLaunchRegs).
-constexpr int kTcLaunchRegs = 168, kTcRegsIo = 72, kTcRegsSoftmax = 216;
-static_assert(128 * kTcRegsIo + 256 * kTcRegsSoftmax <= kTcThreads * kTcLaunchRegs, "register split");
+constexpr int kTcLaunchRegs = 96, kTcRegsIo = 80, kTcRegsSoftmax = 96;
+static_assert(128 * kTcRegsIo + kTcSoftmaxThreads * kTcRegsSoftmax <= kTcThreads * kTcLaunchRegs, "register split");
 constexpr int kTcMaxSlots = 10;
 
 template <int D>
@@ -63,8 +66,8 @@ struct PrefillCfg {
   static constexpr int kAtomBytes = kTcBlockM * 128;    // 128 rows x 128 bytes
   static constexpr int kTileBytes = kTcBlockM * D * 2;  // one 128-row tile of Q, K or V
   static constexpr int kSlots = D == 128 ? 5 : 10;
-  static constexpr int kCtrlBytes = 2048;               // barriers + slack to 1024-align the tiles
-  static constexpr int kSmemBytes = kCtrlBytes + (2 + kSlots) * kTileBytes;
+  static constexpr int kTilesBytes = (2 + kSlots) * kTileBytes;  // at the (1024-aligned) base
+  static constexpr int kSmemBytes = kTilesBytes + 3072;           // + barriers and the row-max exchange
   static_assert(kSlots <= kTcMaxSlots, "slot count");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -76,6 +79,7 @@ struct PrefillCtrl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  float xchg[2][2][kTcBlockM];  // (query tile, column half, row): partial row max / sum
 };
 
 // Wait-site codes reported in the workspace on a timeout.
@@ -157,13 +161,13 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// Row maximum of the 128 scores of a tile (keys >= lim excluded when MASKED),
-// four independent chains of three-input maxima.
-template <bool MASKED>
-__device__ __forceinline__ float row_max(const uint32_t (&sr)[128], int lim) {
+// Row maximum of N scores (keys >= lim excluded when MASKED), four
+// independent chains of three-input maxima.
+template <bool MASKED, int N>
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[N], int lim) {
   float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int q = 0; q < 128; q += 2) {
+  for (int q = 0; q < N; q += 2) {
     float a = __uint_as_float(sr[q]), b = __uint_as_float(sr[q + 1]);
     if (MASKED) {
       a = q < lim ? a : -INFINITY;
@@ -174,17 +178,17 @@ __device__ __forceinline__ float row_max(const uint32_t (&sr)[128], int lim) {
   return fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
 }
 
-// P = 2^(c*s - base) for the 128 scores, written into TMEM over S as packed
-// 16-bit pairs; returns the fp32 row sum.  Score pairs go through the packed
-// fp32x2 FMA; three of every eight pairs are exponentiated by the FMA-pipe
-// polynomial, the rest by the multi-function unit.
-template <bool MASKED, bool BF16>
-__device__ __forceinline__ float exp_store(const uint32_t (&sr)[128], int lim, float c, float base, uint32_t taddr) {
+// P = 2^(c*s - base) for N scores, written into TMEM at taddr as packed
+// 16-bit pairs (N/2 columns); returns the fp32 sum.  Score pairs go through
+// the packed fp32x2 FMA; three of every eight pairs are exponentiated by the
+// FMA-pipe polynomial, the rest by the multi-function unit.
+template <bool MASKED, bool BF16, int N>
+__device__ __forceinline__ float exp_store(const uint32_t (&sr)[N], int lim, float c, float base, uint32_t taddr) {
   const uint64_t c2 = pk2(__float_as_uint(c), __float_as_uint(c));
   const uint64_t nb2 = pk2(__float_as_uint(-base), __float_as_uint(-base));
   uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < N / 32; ++q) {
     uint32_t pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -217,15 +221,24 @@ __device__ __forceinline__ float exp_store(const uint32_t (&sr)[128], int lim, f
   return lo + hi;
 }
 
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
   using Cfg = PrefillCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  PrefillCtrl *ctrl = reinterpret_cast<PrefillCtrl *>(smem_raw);
-  const uint32_t raw_u32 = smem_u32(smem_raw);
-  const uint32_t tiles_u32 = (raw_u32 + 1024u + 1023u) & ~1023u;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The 128B-swizzled tiles need a 1024-byte aligned base; the dynamic shared
+  // memory of a kernel without static shared memory starts aligned.
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) report_error(p.hdr, 2u /* MXFA_ERR_UNSUPPORTED */, 0x1FF);
+    return;
+  }
+  PrefillCtrl *ctrl = reinterpret_cast<PrefillCtrl *>(smem_raw + Cfg::kTilesBytes);
+  const uint32_t tiles_u32 = smem_u32(smem_raw);
   const uint32_t q_u32 = tiles_u32;                              // 2 query tiles
   const uint32_t ring_u32 = tiles_u32 + 2 * Cfg::kTileBytes;     // kSlots KV slots
 
@@ -246,9 +259,9 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&ctrl->s_full[t]), 1);
-      mbar_init(smem_u32(&ctrl->p_full[t]), 4 * 32);
+      mbar_init(smem_u32(&ctrl->p_full[t]), kTcSoftmaxThreads / 2);
       mbar_init(smem_u32(&ctrl->o_done[t]), 1);
-      mbar_init(smem_u32(&ctrl->o_empty[t]), 4 * 32);
+      mbar_init(smem_u32(&ctrl->o_empty[t]), kTcSoftmaxThreads / 2);
     }
     mbar_init(smem_u32(&ctrl->drain), 1);
     ctrl->abort = 0;
@@ -326,23 +339,28 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       constexpr uint32_t idesc_s = make_idesc_f16(BF16, kTcBlockM, kTcBlockN, false, false);
       constexpr uint32_t idesc_o = make_idesc_f16(BF16, kTcBlockM, D, false, true);
       uint32_t ring = 0, p_cnt[2] = {0, 0}, o_uses[2] = {0, 0};
+      // Descriptors are built once per tile; a K-step only moves the start
+      // address (bits 0-13, in 16-byte units), which never carries out.
+      const uint64_t q_desc0 = make_sdesc_sw128(q_u32, 16, 1024);
+      const uint64_t ring_desc0 = make_sdesc_sw128(ring_u32, 16, 1024);
+      const uint64_t v_desc0 = make_sdesc_sw128(ring_u32, Cfg::kAtomBytes, 1024);
+      const uint32_t s_tm[2] = {tmem, tmem + kTcBlockN};
+      const uint32_t o_tm[2] = {tmem + 2 * kTcBlockN, tmem + 2 * kTcBlockN + D};
       auto issue_s = [&](int t, int slot) {
-        const uint32_t qa = q_u32 + t * Cfg::kTileBytes, ka = ring_u32 + slot * Cfg::kTileBytes;
+        const uint64_t qd = q_desc0 + (uint64_t)((t * Cfg::kTileBytes) >> 4);
+        const uint64_t kd = ring_desc0 + (uint64_t)((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Cfg::kAtomBytes + (kk & 3) * 32;
-          mma_ss(tmem + t * kTcBlockN, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)((((kk >> 2) * Cfg::kAtomBytes) + (kk & 3) * 32) >> 4);
+          mma_ss(s_tm[t], qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         mma_commit(smem_u32(&ctrl->s_full[t]));
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
-        const uint32_t va = ring_u32 + slot * Cfg::kTileBytes;
+        const uint64_t vd = v_desc0 + (uint64_t)((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kTcBlockN / 16; ++kk) {
-          mma_ts(tmem + 2 * kTcBlockN + t * D, tmem + t * kTcBlockN + kk * 8,
-                 make_sdesc_sw128(va + kk * 16 * 128, Cfg::kAtomBytes, 1024), idesc_o, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kTcBlockN / 16; ++kk)
+          mma_ts(o_tm[t], s_tm[t] + kk * 8, vd + (uint64_t)(kk * 128), idesc_o, (acc || kk > 0) ? 1u : 0u);
         mma_commit(smem_u32(&ctrl->o_done[t]));
       };
       int it = 0;
@@ -429,15 +447,19 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
   } else {
     regs_inc<kTcRegsSoftmax>();
     // ------------------------------------------------------------ softmax / epilogue
-    const int t = (warp - 4) >> 2;
+    const int t = (warp - 4) >> 3;         // query tile
+    const int ch = ((warp - 4) >> 2) & 1;  // column half
     const int sub = warp & 3;
     const int r = sub * 32 + lane;
+    const int bar_id = 1 + t * 4 + sub;    // the two warps of this row block
     const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16);
-    const uint32_t s_col = t * kTcBlockN, o_col = 2 * kTcBlockN + t * D;
+    const uint32_t s_col = t * kTcBlockN, o_col = 2 * kTcBlockN + t * D + ch * (D / 2);
     const bool neg = p.scale_log2 < 0.f;
     const float cpos = neg ? -p.scale_log2 : p.scale_log2;
     const uint32_t b_s = smem_u32(&ctrl->s_full[t]), b_p = smem_u32(&ctrl->p_full[t]);
     const uint32_t b_od = smem_u32(&ctrl->o_done[t]), b_oe = smem_u32(&ctrl->o_empty[t]);
+    float *x_mine = &ctrl->xchg[t][ch][r];
+    const float *x_other = &ctrl->xchg[t][ch ^ 1][r];
     uint32_t s_cnt = 0, pv_cnt = 0;
     int it = 0;
     bool ok = true;
@@ -457,15 +479,20 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         }
         ++s_cnt;
         tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld128(trow + s_col, sr);
+        uint32_t sr[64];
+        tmem_ld64(trow + s_col + ch * 64, sr);
         if (neg) {  // c*s = (-c)*(-s): fold a negative scale into the scores once
 #pragma unroll
-          for (int q = 0; q < 128; ++q) sr[q] ^= 0x80000000u;
+          for (int q = 0; q < 64; ++q) sr[q] ^= 0x80000000u;
         }
-        const int lim = nv - j * kTcBlockN;  // keys [0, lim) of this tile are visible
-        const bool masked = __any_sync(0xffffffffu, lim < kTcBlockN);
-        const float ext = masked ? row_max<true>(sr, lim) : row_max<false>(sr, lim);
+        const int lim = nv - j * kTcBlockN - ch * 64;  // keys [0, lim) of this half are visible
+        const bool masked = __any_sync(0xffffffffu, lim < 64);
+        float ext = masked ? row_max<true, 64>(sr, lim) : row_max<false, 64>(sr, lim);
+        // swap partial maxima with the other half of the row
+        *x_mine = ext;
+        named_bar_sync(bar_id, 64);
+        ext = fmaxf(ext, *x_other);
+        named_bar_sync(bar_id, 64);  // both have read before either writes again
         const float m_tile = (ext == -INFINITY) ? -INFINITY : ext * cpos;
         const float m_new = fmaxf(m_used, m_tile);
         float alpha = 1.f;
@@ -478,8 +505,8 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
           need = true;
         }
         const float base = (m_used == -INFINITY) ? 0.f : m_used;
-        const float rsum = masked ? exp_store<true, BF16>(sr, lim, cpos, base, trow + s_col)
-                                  : exp_store<false, BF16>(sr, lim, cpos, base, trow + s_col);
+        const float rsum = masked ? exp_store<true, BF16, 64>(sr, lim, cpos, base, trow + s_col + ch * 32)
+                                  : exp_store<false, BF16, 64>(sr, lim, cpos, base, trow + s_col + ch * 32);
         l = l * alpha + rsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // PV_t(j-1) is the latest accumulation into O_t; it must be done.
@@ -491,7 +518,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
           }
           tc_fence_after();
 #pragma unroll
-          for (int q = 0; q < D / 32; ++q) {
+          for (int q = 0; q < D / 64; ++q) {
             uint32_t ov[32];
             tmem_ld32(trow + o_col + q * 32, ov);
 #pragma unroll
@@ -505,8 +532,13 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         ++pv_cnt;
       }
       if (!ok) break;
+      // row sum over both halves
+      *x_mine = l;
+      named_bar_sync(bar_id, 64);
+      l += *x_other;
+      named_bar_sync(bar_id, 64);
       using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-      T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(ui.sr.q0 + i) * p.o_rs + (int64_t)ui.h * p.o_hs;
+      T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(ui.sr.q0 + i) * p.o_rs + (int64_t)ui.h * p.o_hs + ch * (D / 2);
       if (n > 0) {
         const bool got_o = wait_bar(b_od, (pv_cnt - 1) & 1, abort_flag, hdr, kSiteODone);
         __syncwarp();
@@ -514,7 +546,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
+        for (int q = 0; q < D / 64; ++q) {
           uint32_t ov[32];
           tmem_ld32(trow + o_col + q * 32, ov);
           uint32_t pk[16];
@@ -534,9 +566,9 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       } else if (valid) {
         uint4 *dst = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
-        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
+        for (int e = 0; e < D / 16; ++e) dst[e] = make_uint4(0, 0, 0, 0);
       }
-      if (valid && p.lse) {
+      if (valid && ch == 0 && p.lse) {
         p.lse[(int64_t)(ui.sr.q0 + i) * p.hq + ui.h] =
             l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
       }
