@@ -306,23 +306,26 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       const uint32_t s_tmem = tmem + (16u << 16);  // S chains and Q: lanes 16-31 of each sub-partition
       uint32_t tc = 0, g = 0, o_uses = 0;
       bool ok = true;
-      // Descriptors are built once; a chunk / K-step only moves the start
-      // address (bits 0-13, in 16-byte units), which never carries out.
-      const uint64_t k_desc0 = make_sdesc_sw128(ring_u32, 16, 1024);
-      const uint64_t v_desc0 = make_sdesc_sw128(ring_u32, kDcChunkBytes, 1024);
-      const uint64_t p_desc = make_sdesc_sw128(p_u32, 16, 1024);
+      // Descriptors: the high halves are fixed, a chunk / K-step only moves
+      // the start address in the low half (16-byte units, never carries).
+      const uint32_t k_hi = desc_hi(make_sdesc_sw128(ring_u32, 16, 1024));
+      const uint32_t k_lo0 = desc_lo(make_sdesc_sw128(ring_u32, 16, 1024));
+      const uint32_t v_hi = desc_hi(make_sdesc_sw128(ring_u32, kDcChunkBytes, 1024));
+      const uint32_t v_lo0 = desc_lo(make_sdesc_sw128(ring_u32, kDcChunkBytes, 1024));
+      const uint32_t p_hi = desc_hi(make_sdesc_sw128(p_u32, 16, 1024));
+      const uint32_t p_lo0 = desc_lo(make_sdesc_sw128(p_u32, 16, 1024));
       // S of tile counter `t` into the three chains (chunk c accumulates into chain c % 3).
       auto issue_s = [&](uint32_t t) -> bool {
         const int x = t % kDcRingTiles;
         if (!wait_bar(b_tf(x), (t / kDcRingTiles) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
         tc_fence_after();
-        const uint64_t kd = k_desc0 + (uint64_t)((x * kDcChunks * kDcChunkBytes) >> 4);
+        const uint32_t k_lo = k_lo0 + (uint32_t)((x * kDcChunks * kDcChunkBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
           for (int c = 0; c < kDcChunks; ++c)
-            mma_ts(s_tmem + (c % 3) * kDcKeys, s_tmem + kDcQCol + (c * 4 + kk) * 8,
-                   kd + (uint64_t)((c * kDcChunkBytes + kk * 32) >> 4), idesc_s, (c >= 3 || kk > 0) ? 1u : 0u);
+            mma_ts2(s_tmem + (c % 3) * kDcKeys, s_tmem + kDcQCol + (c * 4 + kk) * 8,
+                    k_lo + (uint32_t)((c * kDcChunkBytes + kk * 32) >> 4), k_hi, idesc_s, (c >= 3 || kk > 0) ? 1u : 0u);
         mma_commit(b_sf);
         return true;
       };
@@ -350,14 +353,14 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
             break;
           }
           tc_fence_after();
-          const uint64_t vd = v_desc0 + (uint64_t)(((tc % kDcRingTiles) * kDcChunks * kDcChunkBytes) >> 4);
+          const uint32_t v_lo = v_lo0 + (uint32_t)(((tc % kDcRingTiles) * kDcChunks * kDcChunkBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
             for (int half = 0; half < 2; ++half)
-              mma_ss(tmem + half * 256, p_desc + (uint64_t)(kk * 2),
-                     vd + (uint64_t)((half * 4 * kDcChunkBytes + kk * 16 * 128) >> 4), idesc_o,
-                     (jj > 0 || kk > 0) ? 1u : 0u);
+              mma_ss2(tmem + half * 256, p_lo0 + (uint32_t)(kk * 2), p_hi,
+                      v_lo + (uint32_t)((half * 4 * kDcChunkBytes + kk * 16 * 128) >> 4), v_hi, idesc_o,
+                      (jj > 0 || kk > 0) ? 1u : 0u);
           mma_commit(b_od);
           mma_commit(b_te(tc % kDcRingTiles));
         }

@@ -254,7 +254,8 @@ mxfa_status_t launch_tc(const AttnParams &p, const CUtensorMap &mq, const CUtens
   int sms = 0;
   MXFA_TRY(sm_count(&sms));
   auto k = attn_fwd_tc_kernel<D, BF16>;
-  MXFA_TRY(check_launch_regs(reinterpret_cast<const void *>(k), kTcLaunchRegs));
+  if (kTcRegsIo != kTcLaunchRegs || kTcRegsSoftmax != kTcLaunchRegs)  // a setmaxnreg split is compiled in
+    MXFA_TRY(check_launch_regs(reinterpret_cast<const void *>(k), kTcLaunchRegs));
   MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(k), PrefillCfg<D>::kSmemBytes));
   k<<<sms, kTcThreads, PrefillCfg<D>::kSmemBytes, st>>>(p, mq, mk, mv);
   MXFA_CUDA(cudaGetLastError());

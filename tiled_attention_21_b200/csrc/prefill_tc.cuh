@@ -6,9 +6,11 @@
 // (128 keys) and query tile t:
 //     S_t  = Q_t K_j^T           tcgen05.mma, A = Q (smem), B = K (smem),
 //                                fp32 accumulator in TMEM
-//     P_t  = exp2(c*S_t - m)     softmax warpgroup t, one thread per row,
-//                                c = softmax_scale*log2(e); P written back
-//                                into TMEM over S_t as bf16/f16
+//     P_t  = exp2(c*S_t - m)     softmax, two threads per row (one per
+//                                64-key half), c = softmax_scale*log2(e);
+//                                P written back into TMEM over S_t as
+//                                bf16/f16 (keys 0-63 in columns 0-31,
+//                                keys 64-127 in columns 64-95)
 //     O_t += P_t V_j             tcgen05.mma, A = P (TMEM), B = V (smem)
 // The online-softmax bookkeeping follows mxflashattn 1.4.0 prefill.py
 // (prefill_chunked_reference: running max, correction of the accumulator,
@@ -51,12 +53,13 @@ constexpr int kTcBlockN = 128;  // keys per KV tile
 constexpr int kTcUnitRows = 2 * kTcBlockM;
 constexpr int kTcThreads = 640;
 constexpr int kTcSoftmaxThreads = 512;  // four warpgroups: (query tile, column half)
-// Register split (setmaxnreg): launched at kTcLaunchRegs per thread, the
-// producer/MMA warpgroup drops to kTcRegsIo and the four softmax warpgroups
-// rise to kTcRegsSoftmax; 128*kTcRegsIo + 512*kTcRegsSoftmax must not exceed
-// 640*kTcLaunchRegs (the host refuses to launch a build whose register count
-// differs from kTcLaunchRegs).
-constexpr int kTcLaunchRegs = 96, kTcRegsIo = 80, kTcRegsSoftmax = 96;
+// Register budgets: launched at kTcLaunchRegs per thread; if the budgets of
+// the producer/MMA warpgroup (kTcRegsIo) and of the four softmax warpgroups
+// (kTcRegsSoftmax) differ, setmaxnreg moves registers between them, and
+// 128*kTcRegsIo + 512*kTcRegsSoftmax must not exceed 640*kTcLaunchRegs (the
+// host refuses to launch a build whose register count differs from
+// kTcLaunchRegs).  The softmax reads S in 32-column pieces so both fit in 96.
+constexpr int kTcLaunchRegs = 96, kTcRegsIo = 96, kTcRegsSoftmax = 96;
 static_assert(128 * kTcRegsIo + kTcSoftmaxThreads * kTcRegsSoftmax <= kTcThreads * kTcLaunchRegs, "register split");
 constexpr int kTcMaxSlots = 10;
 
@@ -285,7 +288,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
   const int grid = gridDim.x, cta = blockIdx.x;
 
   if (warp < 4) {
-  regs_dec<kTcRegsIo>();
+  if constexpr (kTcRegsIo != kTcLaunchRegs) regs_dec<kTcRegsIo>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -339,28 +342,29 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       constexpr uint32_t idesc_s = make_idesc_f16(BF16, kTcBlockM, kTcBlockN, false, false);
       constexpr uint32_t idesc_o = make_idesc_f16(BF16, kTcBlockM, D, false, true);
       uint32_t ring = 0, p_cnt[2] = {0, 0}, o_uses[2] = {0, 0};
-      // Descriptors are built once per tile; a K-step only moves the start
-      // address (bits 0-13, in 16-byte units), which never carries out.
-      const uint64_t q_desc0 = make_sdesc_sw128(q_u32, 16, 1024);
-      const uint64_t ring_desc0 = make_sdesc_sw128(ring_u32, 16, 1024);
-      const uint64_t v_desc0 = make_sdesc_sw128(ring_u32, Cfg::kAtomBytes, 1024);
+      // Descriptors: the high halves are fixed, a K-step only moves the
+      // start address in the low half (16-byte units, never carries).
+      const uint32_t sd_hi = desc_hi(make_sdesc_sw128(q_u32, 16, 1024));
+      const uint32_t vd_hi = desc_hi(make_sdesc_sw128(ring_u32, Cfg::kAtomBytes, 1024));
+      const uint32_t ring_lo = desc_lo(make_sdesc_sw128(ring_u32, 16, 1024));
+      const uint32_t vring_lo = desc_lo(make_sdesc_sw128(ring_u32, Cfg::kAtomBytes, 1024));
+      const uint32_t q_lo0 = desc_lo(make_sdesc_sw128(q_u32, 16, 1024));
       const uint32_t s_tm[2] = {tmem, tmem + kTcBlockN};
       const uint32_t o_tm[2] = {tmem + 2 * kTcBlockN, tmem + 2 * kTcBlockN + D};
       auto issue_s = [&](int t, int slot) {
-        const uint64_t qd = q_desc0 + (uint64_t)((t * Cfg::kTileBytes) >> 4);
-        const uint64_t kd = ring_desc0 + (uint64_t)((slot * Cfg::kTileBytes) >> 4);
+        const uint32_t k_lo = ring_lo + (uint32_t)((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)((((kk >> 2) * Cfg::kAtomBytes) + (kk & 3) * 32) >> 4);
-          mma_ss(s_tm[t], qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss2(s_tm[t], q_lo0 + (uint32_t)((t * Cfg::kTileBytes + (kk >> 2) * Cfg::kAtomBytes + (kk & 3) * 32) >> 4), sd_hi,
+                  k_lo + (uint32_t)((((kk >> 2) * Cfg::kAtomBytes) + (kk & 3) * 32) >> 4), sd_hi, idesc_s, kk > 0 ? 1u : 0u);
         mma_commit(smem_u32(&ctrl->s_full[t]));
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
-        const uint64_t vd = v_desc0 + (uint64_t)((slot * Cfg::kTileBytes) >> 4);
+        const uint32_t v_lo = vring_lo + (uint32_t)((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kTcBlockN / 16; ++kk)
-          mma_ts(o_tm[t], s_tm[t] + kk * 8, vd + (uint64_t)(kk * 128), idesc_o, (acc || kk > 0) ? 1u : 0u);
+          mma_ts2(o_tm[t], s_tm[t] + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), v_lo + (uint32_t)(kk * 128), vd_hi, idesc_o,
+                  (acc || kk > 0) ? 1u : 0u);
         mma_commit(smem_u32(&ctrl->o_done[t]));
       };
       int it = 0;
@@ -445,7 +449,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     }
   }
   } else {
-    regs_inc<kTcRegsSoftmax>();
+    if constexpr (kTcRegsSoftmax != kTcLaunchRegs) regs_inc<kTcRegsSoftmax>();
     // ------------------------------------------------------------ softmax / epilogue
     const int t = (warp - 4) >> 3;         // query tile
     const int ch = ((warp - 4) >> 2) & 1;  // column half
@@ -479,15 +483,20 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         }
         ++s_cnt;
         tc_fence_after();
-        uint32_t sr[64];
-        tmem_ld64(trow + s_col + ch * 64, sr);
-        if (neg) {  // c*s = (-c)*(-s): fold a negative scale into the scores once
-#pragma unroll
-          for (int q = 0; q < 64; ++q) sr[q] ^= 0x80000000u;
-        }
+        // pass 1: maximum of this thread's 64 scores, 32 columns at a time
+        const uint32_t s_addr = trow + s_col + ch * 64;
         const int lim = nv - j * kTcBlockN - ch * 64;  // keys [0, lim) of this half are visible
         const bool masked = __any_sync(0xffffffffu, lim < 64);
-        float ext = masked ? row_max<true, 64>(sr, lim) : row_max<false, 64>(sr, lim);
+        const uint32_t flip = neg ? 0x80000000u : 0u;  // c*s = (-c)*(-s) folds a negative scale
+        float ext = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t sa[32];
+          tmem_ld32(s_addr + q * 32, sa);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sa[e] ^= flip;
+          ext = fmaxf(ext, masked ? row_max<true, 32>(sa, lim - q * 32) : row_max<false, 32>(sa, lim - q * 32));
+        }
         // swap partial maxima with the other half of the row
         *x_mine = ext;
         named_bar_sync(bar_id, 64);
@@ -505,8 +514,18 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
           need = true;
         }
         const float base = (m_used == -INFINITY) ? 0.f : m_used;
-        const float rsum = masked ? exp_store<true, BF16, 64>(sr, lim, cpos, base, trow + s_col + ch * 32)
-                                  : exp_store<false, BF16, 64>(sr, lim, cpos, base, trow + s_col + ch * 32);
+        // pass 2: P = 2^(c*s - base), 32 columns at a time, written over this
+        // thread's own S columns (keys 0-63 -> columns 0-31, 64-127 -> 64-95)
+        float rsum = 0.f;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t sa[32];
+          tmem_ld32(s_addr + q * 32, sa);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sa[e] ^= flip;
+          rsum += masked ? exp_store<true, BF16, 32>(sa, lim - q * 32, cpos, base, s_addr + q * 16)
+                         : exp_store<false, BF16, 32>(sa, lim - q * 32, cpos, base, s_addr + q * 16);
+        }
         l = l * alpha + rsum;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // PV_t(j-1) is the latest accumulation into O_t; it must be done.
