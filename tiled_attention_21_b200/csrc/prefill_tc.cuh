@@ -82,7 +82,7 @@ struct PrefillCtrl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  float xchg[2][2][kTcBlockM];  // (query tile, column half, row): partial row max / sum
+  float xchg[4][kTcBlockM];  // (column group, row): partial row max / sum
 };
 
 // Wait-site codes reported in the workspace on a timeout.
@@ -145,6 +145,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 __device__ __forceinline__ uint64_t pk2(uint32_t lo, uint32_t hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
@@ -164,21 +169,23 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// Row maximum of N scores (keys >= lim excluded when MASKED), four
-// independent chains of three-input maxima.
-template <bool MASKED, int N>
-__device__ __forceinline__ float row_max(const uint32_t (&sr)[N], int lim) {
-  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+// Largest (NEG: smallest) of N scores, keys >= lim excluded when MASKED
+// (an empty set gives -inf, NEG: +inf); four independent chains of
+// three-input maxima / minima.
+template <bool MASKED, bool NEG, int N>
+__device__ __forceinline__ float row_ext(const uint32_t (&sr)[N], int lim) {
+  constexpr float kEmpty = NEG ? INFINITY : -INFINITY;
+  float m4[4] = {kEmpty, kEmpty, kEmpty, kEmpty};
 #pragma unroll
   for (int q = 0; q < N; q += 2) {
     float a = __uint_as_float(sr[q]), b = __uint_as_float(sr[q + 1]);
     if (MASKED) {
-      a = q < lim ? a : -INFINITY;
-      b = q + 1 < lim ? b : -INFINITY;
+      a = q < lim ? a : kEmpty;
+      b = q + 1 < lim ? b : kEmpty;
     }
-    m4[(q >> 1) & 3] = fmax3(m4[(q >> 1) & 3], a, b);
+    m4[(q >> 1) & 3] = NEG ? fmin3(m4[(q >> 1) & 3], a, b) : fmax3(m4[(q >> 1) & 3], a, b);
   }
-  return fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+  return NEG ? fmin3(fminf(m4[0], m4[1]), m4[2], m4[3]) : fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
 }
 
 // P = 2^(c*s - base) for N scores, written into TMEM at taddr as packed
@@ -227,6 +234,24 @@ __device__ __forceinline__ float exp_store(const uint32_t (&sr)[N], int lim, flo
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Named barrier that also returns the AND (bar_and) or OR (bar_or) of a
+// per-thread predicate over the `count` participating threads.
+__device__ __forceinline__ bool bar_and(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile("{\n .reg .pred q, p;\n setp.ne.u32 q, %1, 0;\n bar.red.and.pred p, %2, %3, q;\n selp.u32 %0, 1, 0, p;\n}\n"
+               : "=r"(r)
+               : "r"((uint32_t)v), "r"(id), "r"(count)
+               : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool bar_or(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile("{\n .reg .pred q, p;\n setp.ne.u32 q, %1, 0;\n bar.red.or.pred p, %2, %3, q;\n selp.u32 %0, 1, 0, p;\n}\n"
+               : "=r"(r)
+               : "r"((uint32_t)v), "r"(id), "r"(count)
+               : "memory");
+  return r != 0;
+}
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -262,9 +287,9 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&ctrl->s_full[t]), 1);
-      mbar_init(smem_u32(&ctrl->p_full[t]), kTcSoftmaxThreads / 2);
+      mbar_init(smem_u32(&ctrl->p_full[t]), kTcSoftmaxThreads / 32);  // one arrival per softmax warp
       mbar_init(smem_u32(&ctrl->o_done[t]), 1);
-      mbar_init(smem_u32(&ctrl->o_empty[t]), kTcSoftmaxThreads / 2);
+      mbar_init(smem_u32(&ctrl->o_empty[t]), kTcSoftmaxThreads / 32);
     }
     mbar_init(smem_u32(&ctrl->drain), 1);
     ctrl->abort = 0;
@@ -363,7 +388,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         const uint32_t v_lo = vring_lo + (uint32_t)((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kTcBlockN / 16; ++kk)
-          mma_ts2(o_tm[t], s_tm[t] + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), v_lo + (uint32_t)(kk * 128), vd_hi, idesc_o,
+          mma_ts2(o_tm[t], s_tm[t] + (kk >> 1) * 32 + (kk & 1) * 8, v_lo + (uint32_t)(kk * 128), vd_hi, idesc_o,
                   (acc || kk > 0) ? 1u : 0u);
         mma_commit(smem_u32(&ctrl->o_done[t]));
       };
@@ -451,145 +476,155 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
   } else {
     if constexpr (kTcRegsSoftmax != kTcLaunchRegs) regs_inc<kTcRegsSoftmax>();
     // ------------------------------------------------------------ softmax / epilogue
-    const int t = (warp - 4) >> 3;         // query tile
-    const int ch = ((warp - 4) >> 2) & 1;  // column half
+    // Four threads per query row, one per 32-key column group g; the four
+    // warps of a TMEM sub-partition take both query tiles in turn, so every
+    // score is read from TMEM once and stays in registers.
+    const int g = (warp - 4) >> 2;  // column group: keys [32g, 32g+32), output columns [g*D/4, (g+1)*D/4)
     const int sub = warp & 3;
     const int r = sub * 32 + lane;
-    const int bar_id = 1 + t * 4 + sub;    // the two warps of this row block
+    const int bar_id = 1 + sub;     // the four warps of this sub-partition
+    constexpr int OC = D / 4;       // output columns per thread
     const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16);
-    const uint32_t s_col = t * kTcBlockN, o_col = 2 * kTcBlockN + t * D + ch * (D / 2);
     const bool neg = p.scale_log2 < 0.f;
-    const float cpos = neg ? -p.scale_log2 : p.scale_log2;
-    const uint32_t b_s = smem_u32(&ctrl->s_full[t]), b_p = smem_u32(&ctrl->p_full[t]);
-    const uint32_t b_od = smem_u32(&ctrl->o_done[t]), b_oe = smem_u32(&ctrl->o_empty[t]);
-    float *x_mine = &ctrl->xchg[t][ch][r];
-    const float *x_other = &ctrl->xchg[t][ch ^ 1][r];
-    uint32_t s_cnt = 0, pv_cnt = 0;
+    const float c = p.scale_log2;
+    float *x_mine = &ctrl->xchg[g][r];
+    uint32_t s_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
     int it = 0;
     bool ok = true;
     for (int u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
       const UnitInfo ui = unit_info(p, u);
-      const int n = ui.n[t];
-      const int i = ui.m * kTcUnitRows + t * kTcBlockM + r;
-      const bool valid = i < ui.sr.sq;
-      const int nv = valid ? visible_keys(i, ui.sr.sq, ui.sr.sk, p.causal) : 0;
-      float m_used = -INFINITY, l = 0.f;
-      for (int j = 0; j < n; ++j) {
-        const bool got_s = wait_bar(b_s, s_cnt & 1, abort_flag, hdr, kSiteSFull);
+      const int nmax = max(ui.n[0], ui.n[1]);
+      int i[2], nv[2];
+      float m_used[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        i[t] = ui.m * kTcUnitRows + t * kTcBlockM + r;
+        nv[t] = i[t] < ui.sr.sq ? visible_keys(i[t], ui.sr.sq, ui.sr.sk, p.causal) : 0;
+      }
+      for (int j = 0; j < nmax && ok; ++j) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (j >= ui.n[t]) continue;
+          // A failed wait does not leave the loop here: the four warps of the
+          // sub-partition first agree on it at the next named barrier, so
+          // none is left waiting there for a warp that has gone.
+          const bool got_s = wait_bar(smem_u32(&ctrl->s_full[t]), s_cnt[t] & 1, abort_flag, hdr, kSiteSFull);
+          __syncwarp();
+          const bool wok = __all_sync(0xffffffffu, got_s);
+          ++s_cnt[t];
+          tc_fence_after();
+          const uint32_t s_addr = trow + t * kTcBlockN + g * 32;
+          const int lim = nv[t] - j * kTcBlockN - g * 32;  // keys [0, lim) of this group are visible
+          const bool masked = __any_sync(0xffffffffu, lim < 32);
+          uint32_t sa[32];
+          tmem_ld32(s_addr, sa);
+          // this group's largest c*s (a negative c turns the largest into the smallest s)
+          const float ext = neg ? (masked ? row_ext<true, true, 32>(sa, lim) : row_ext<false, true, 32>(sa, lim))
+                                : (masked ? row_ext<true, false, 32>(sa, lim) : row_ext<false, false, 32>(sa, lim));
+          const float pm = (ext == (neg ? INFINITY : -INFINITY)) ? -INFINITY : ext * c;
+          float alpha = 1.f;
+          bool need = false;
+          // Fast path: the stale base still bounds every group of every row
+          // of this sub-partition (no row grew by more than 2^8).
+          if (!bar_and(bar_id, 128, wok && m_used[t] != -INFINITY && pm <= m_used[t] + 8.f)) {
+            if (bar_or(bar_id, 128, !wok)) {
+              ok = false;
+              break;
+            }
+            *x_mine = pm;
+            named_bar_sync(bar_id, 128);
+            const float mt = fmaxf(fmaxf(ctrl->xchg[0][r], ctrl->xchg[1][r]), fmaxf(ctrl->xchg[2][r], ctrl->xchg[3][r]));
+            named_bar_sync(bar_id, 128);  // all have read before any writes again
+            const float m_new = fmaxf(m_used[t], mt);
+            if (m_used[t] == -INFINITY) {
+              m_used[t] = m_new;  // nothing accumulated yet
+            } else if (m_new > m_used[t] + 8.f) {
+              alpha = ex2(m_used[t] - m_new);
+              m_used[t] = m_new;
+              need = true;
+            }
+          }
+          const float base = (m_used[t] == -INFINITY) ? 0.f : m_used[t];
+          // P = 2^(c*s - base) written as 16 packed columns at the start of
+          // this group's own S columns
+          const float rsum = masked ? exp_store<true, BF16, 32>(sa, lim, c, base, s_addr)
+                                    : exp_store<false, BF16, 32>(sa, lim, c, base, s_addr);
+          l[t] = l[t] * alpha + rsum;
+          if (j > 0 && __any_sync(0xffffffffu, need)) {
+            // Rescale O_t.  PV_t(j-1), its latest accumulation, is complete:
+            // it was issued before S_t(j), and the commit that signalled
+            // S_t(j) tracks every earlier MMA of the issuing thread.
+            const uint32_t oa = trow + 2 * kTcBlockN + t * D + g * OC;
+            if constexpr (OC == 32) {
+              uint32_t ov[32];
+              tmem_ld32(oa, ov);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+              tmem_st32(oa, ov);
+            } else {
+              uint32_t ov[16];
+              tmem_ld16(oa, ov);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+              tmem_st16(oa, ov);
+            }
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&ctrl->p_full[t]));
+          ++pv_cnt[t];
+        }
+      }
+      if (!ok) break;
+      // epilogue of both query tiles
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        bool got_o = true;
+        if (ui.n[t] > 0) got_o = wait_bar(smem_u32(&ctrl->o_done[t]), (pv_cnt[t] - 1) & 1, abort_flag, hdr, kSiteODone);
         __syncwarp();
-        if (!__all_sync(0xffffffffu, got_s)) {
+        if (bar_or(bar_id, 128, !__all_sync(0xffffffffu, got_o))) {
           ok = false;
           break;
         }
-        ++s_cnt;
-        tc_fence_after();
-        // pass 1: maximum of this thread's 64 scores, 32 columns at a time
-        const uint32_t s_addr = trow + s_col + ch * 64;
-        const int lim = nv - j * kTcBlockN - ch * 64;  // keys [0, lim) of this half are visible
-        const bool masked = __any_sync(0xffffffffu, lim < 64);
-        const uint32_t flip = neg ? 0x80000000u : 0u;  // c*s = (-c)*(-s) folds a negative scale
-        float ext = -INFINITY;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t sa[32];
-          tmem_ld32(s_addr + q * 32, sa);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) sa[e] ^= flip;
-          ext = fmaxf(ext, masked ? row_max<true, 32>(sa, lim - q * 32) : row_max<false, 32>(sa, lim - q * 32));
-        }
-        // swap partial maxima with the other half of the row
-        *x_mine = ext;
-        named_bar_sync(bar_id, 64);
-        ext = fmaxf(ext, *x_other);
-        named_bar_sync(bar_id, 64);  // both have read before either writes again
-        const float m_tile = (ext == -INFINITY) ? -INFINITY : ext * cpos;
-        const float m_new = fmaxf(m_used, m_tile);
-        float alpha = 1.f;
-        bool need = false;
-        if (m_used == -INFINITY) {
-          m_used = m_new;  // nothing accumulated yet
-        } else if (m_new > m_used + 8.f) {
-          alpha = ex2(m_used - m_new);
-          m_used = m_new;
-          need = true;
-        }
-        const float base = (m_used == -INFINITY) ? 0.f : m_used;
-        // pass 2: P = 2^(c*s - base), 32 columns at a time, written over this
-        // thread's own S columns (keys 0-63 -> columns 0-31, 64-127 -> 64-95)
-        float rsum = 0.f;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t sa[32];
-          tmem_ld32(s_addr + q * 32, sa);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) sa[e] ^= flip;
-          rsum += masked ? exp_store<true, BF16, 32>(sa, lim - q * 32, cpos, base, s_addr + q * 16)
-                         : exp_store<false, BF16, 32>(sa, lim - q * 32, cpos, base, s_addr + q * 16);
-        }
-        l = l * alpha + rsum;
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // PV_t(j-1) is the latest accumulation into O_t; it must be done.
-          const bool got_o = wait_bar(b_od, (pv_cnt - 1) & 1, abort_flag, hdr, kSiteODone);
-          __syncwarp();
-          if (!__all_sync(0xffffffffu, got_o)) {
-            ok = false;
-            break;
-          }
+        // row sum over the four groups
+        *x_mine = l[t];
+        named_bar_sync(bar_id, 128);
+        const float lt = (ctrl->xchg[0][r] + ctrl->xchg[1][r]) + (ctrl->xchg[2][r] + ctrl->xchg[3][r]);
+        named_bar_sync(bar_id, 128);
+        const bool valid = i[t] < ui.sr.sq;
+        using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+        T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(ui.sr.q0 + i[t]) * p.o_rs + (int64_t)ui.h * p.o_hs + g * OC;
+        if (ui.n[t] > 0) {
           tc_fence_after();
+          const float inv = lt > 0.f ? 1.f / lt : 0.f;
+          const uint32_t oa = trow + 2 * kTcBlockN + t * D + g * OC;
+          uint32_t ov[OC];
+          if constexpr (OC == 32) tmem_ld32(oa, ov);
+          else tmem_ld16(oa, ov);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&ctrl->o_empty[t]));
+          uint32_t pk[OC / 2];
 #pragma unroll
-          for (int q = 0; q < D / 64; ++q) {
-            uint32_t ov[32];
-            tmem_ld32(trow + o_col + q * 32, ov);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(trow + o_col + q * 32, ov);
-          }
-          tmem_wait_st();
-        }
-        tc_fence_before();
-        mbar_arrive(b_p);
-        ++pv_cnt;
-      }
-      if (!ok) break;
-      // row sum over both halves
-      *x_mine = l;
-      named_bar_sync(bar_id, 64);
-      l += *x_other;
-      named_bar_sync(bar_id, 64);
-      using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-      T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(ui.sr.q0 + i) * p.o_rs + (int64_t)ui.h * p.o_hs + ch * (D / 2);
-      if (n > 0) {
-        const bool got_o = wait_bar(b_od, (pv_cnt - 1) & 1, abort_flag, hdr, kSiteODone);
-        __syncwarp();
-        if (!__all_sync(0xffffffffu, got_o)) break;
-        tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-        for (int q = 0; q < D / 64; ++q) {
-          uint32_t ov[32];
-          tmem_ld32(trow + o_col + q * 32, ov);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
+          for (int e = 0; e < OC / 2; ++e) {
             const float a0 = __uint_as_float(ov[2 * e]) * inv, a1 = __uint_as_float(ov[2 * e + 1]) * inv;
             pk[e] = BF16 ? pack_bf16x2(a0, a1) : pack_f16x2(a0, a1);
           }
           if (valid) {
-            uint4 *dst = reinterpret_cast<uint4 *>(orow + q * 32);
+            uint4 *dst = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            for (int e = 0; e < OC / 8; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
           }
-        }
-        tc_fence_before();
-        mbar_arrive(b_oe);
-      } else if (valid) {
-        uint4 *dst = reinterpret_cast<uint4 *>(orow);
+        } else if (valid) {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
-        for (int e = 0; e < D / 16; ++e) dst[e] = make_uint4(0, 0, 0, 0);
-      }
-      if (valid && ch == 0 && p.lse) {
-        p.lse[(int64_t)(ui.sr.q0 + i) * p.hq + ui.h] =
-            l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+          for (int e = 0; e < OC / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
+        }
+        if (valid && g == 0 && p.lse) {
+          p.lse[(int64_t)(ui.sr.q0 + i[t]) * p.hq + ui.h] =
+              lt > 0.f ? (m_used[t] + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+        }
       }
     }
   }
