@@ -231,6 +231,12 @@ __device__ __forceinline__ float exp_store(const uint32_t (&sr)[N], int lim, flo
   return lo + hi;
 }
 
+// One lane of a converged warp (elect.sync).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t r;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(r));
+  return r != 0;
+}
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
@@ -363,7 +369,14 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the schedule, so MMA operands are computed
+    // warp-uniformly; one elected lane issues each tcgen05 operation.
+    const bool leader = elect_one();
+    // every lane waits; the warp gives up together if any lane gave up
+    auto wait_warp = [&](uint32_t bar, uint32_t parity, volatile int *ab, WsHeader *h, uint32_t site) {
+      return __all_sync(0xffffffffu, wait_bar(bar, parity, ab, h, site));
+    };
+    {
       constexpr uint32_t idesc_s = make_idesc_f16(BF16, kTcBlockM, kTcBlockN, false, false);
       constexpr uint32_t idesc_o = make_idesc_f16(BF16, kTcBlockM, D, false, true);
       uint32_t ring = 0, p_cnt[2] = {0, 0}, o_uses[2] = {0, 0};
@@ -374,49 +387,50 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       const uint32_t ring_lo = desc_lo(make_sdesc_sw128(ring_u32, 16, 1024));
       const uint32_t vring_lo = desc_lo(make_sdesc_sw128(ring_u32, Cfg::kAtomBytes, 1024));
       const uint32_t q_lo0 = desc_lo(make_sdesc_sw128(q_u32, 16, 1024));
-      const uint32_t s_tm[2] = {tmem, tmem + kTcBlockN};
-      const uint32_t o_tm[2] = {tmem + 2 * kTcBlockN, tmem + 2 * kTcBlockN + D};
+      const uint32_t tm_base = __shfl_sync(0xffffffffu, tmem, 0);
+      const uint32_t s_tm[2] = {tm_base, tm_base + kTcBlockN};
+      const uint32_t o_tm[2] = {tm_base + 2 * kTcBlockN, tm_base + 2 * kTcBlockN + D};
       auto issue_s = [&](int t, int slot) {
         const uint32_t k_lo = ring_lo + (uint32_t)((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss2(s_tm[t], q_lo0 + (uint32_t)((t * Cfg::kTileBytes + (kk >> 2) * Cfg::kAtomBytes + (kk & 3) * 32) >> 4), sd_hi,
+          if (leader) mma_ss2(s_tm[t], q_lo0 + (uint32_t)((t * Cfg::kTileBytes + (kk >> 2) * Cfg::kAtomBytes + (kk & 3) * 32) >> 4), sd_hi,
                   k_lo + (uint32_t)((((kk >> 2) * Cfg::kAtomBytes) + (kk & 3) * 32) >> 4), sd_hi, idesc_s, kk > 0 ? 1u : 0u);
-        mma_commit(smem_u32(&ctrl->s_full[t]));
+        if (leader) mma_commit(smem_u32(&ctrl->s_full[t]));
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
         const uint32_t v_lo = vring_lo + (uint32_t)((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kTcBlockN / 16; ++kk)
-          mma_ts2(o_tm[t], s_tm[t] + (kk >> 1) * 32 + (kk & 1) * 8, v_lo + (uint32_t)(kk * 128), vd_hi, idesc_o,
+          if (leader) mma_ts2(o_tm[t], s_tm[t] + (kk >> 1) * 32 + (kk & 1) * 8, v_lo + (uint32_t)(kk * 128), vd_hi, idesc_o,
                   (acc || kk > 0) ? 1u : 0u);
-        mma_commit(smem_u32(&ctrl->o_done[t]));
+        if (leader) mma_commit(smem_u32(&ctrl->o_done[t]));
       };
       int it = 0;
       bool ok = true;
       for (int u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
         const UnitInfo ui = unit_info(p, u);
         const int nmax = max(ui.n[0], ui.n[1]);
-        if (!wait_bar(b_qf, it & 1, abort_flag, hdr, kSiteQFull)) break;
+        if (!wait_warp(b_qf, it & 1, abort_flag, hdr, kSiteQFull)) break;
         tc_fence_after();
         if (nmax == 0) {
-          mma_commit(b_qe);
+          if (leader) mma_commit(b_qe);
           continue;
         }
         // prologue: S_t(0)
         {
           const int ks = ring % Cfg::kSlots;
-          if (!wait_bar(b_sf(ks), (ring / Cfg::kSlots) & 1, abort_flag, hdr, kSiteSlotFull)) break;
+          if (!wait_warp(b_sf(ks), (ring / Cfg::kSlots) & 1, abort_flag, hdr, kSiteSlotFull)) break;
           ++ring;
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
             if (ui.n[t] > 0) issue_s(t, ks);
-          mma_commit(b_se(ks));
-          if (nmax == 1) mma_commit(b_qe);
+          if (leader) mma_commit(b_se(ks));
+          if (nmax == 1 && leader) mma_commit(b_qe);
         }
         for (int j = 0; j < nmax && ok; ++j) {
           const int vs = ring % Cfg::kSlots;
-          if (!wait_bar(b_sf(vs), (ring / Cfg::kSlots) & 1, abort_flag, hdr, kSiteSlotFull)) {
+          if (!wait_warp(b_sf(vs), (ring / Cfg::kSlots) & 1, abort_flag, hdr, kSiteSlotFull)) {
             ok = false;
             break;
           }
@@ -433,13 +447,13 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
           }
           for (int t = 0; t < 2 && ok; ++t) {
             if (j >= ui.n[t]) continue;
-            if (!wait_bar(smem_u32(&ctrl->p_full[t]), p_cnt[t] & 1, abort_flag, hdr, kSitePFull)) {
+            if (!wait_warp(smem_u32(&ctrl->p_full[t]), p_cnt[t] & 1, abort_flag, hdr, kSitePFull)) {
               ok = false;
               break;
             }
             ++p_cnt[t];
             if (j == 0 && o_uses[t] > 0 &&
-                !wait_bar(smem_u32(&ctrl->o_empty[t]), (o_uses[t] - 1) & 1, abort_flag, hdr, kSiteOEmpty)) {
+                !wait_warp(smem_u32(&ctrl->o_empty[t]), (o_uses[t] - 1) & 1, abort_flag, hdr, kSiteOEmpty)) {
               ok = false;
               break;
             }
@@ -447,7 +461,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
             issue_pv(t, vs, j > 0);
             if (j + 1 < ui.n[t]) {
               if (!kwaited) {
-                if (!wait_bar(b_sf(ks), kph, abort_flag, hdr, kSiteSlotFull)) {
+                if (!wait_warp(b_sf(ks), kph, abort_flag, hdr, kSiteSlotFull)) {
                   ok = false;
                   break;
                 }
@@ -458,16 +472,16 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
             }
           }
           if (!ok) break;
-          mma_commit(b_se(vs));
-          if (has_next) mma_commit(b_se(ks));
-          if (j == nmax - 2) mma_commit(b_qe);
+          if (leader) mma_commit(b_se(vs));
+          if (has_next && leader) mma_commit(b_se(ks));
+          if (j == nmax - 2 && leader) mma_commit(b_qe);
         }
         if (!ok) break;
         for (int t = 0; t < 2; ++t)
           if (ui.n[t] > 0) ++o_uses[t];
       }
-      // Teardown: all MMAs issued by this thread complete before TMEM is freed.
-      mma_commit(smem_u32(&ctrl->drain));
+      // Teardown: all MMAs issued by the elected lane complete before TMEM is freed.
+      if (leader) mma_commit(smem_u32(&ctrl->drain));
       const uint64_t t0 = global_ns();
       while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < kWaitBudgetNs) {
       }
