@@ -300,10 +300,18 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the schedule, so MMA operands are computed
+    // warp-uniformly; one elected lane issues each tcgen05 operation, and
+    // the warp gives up a wait together if any lane gave up.
+    const bool leader = elect_one();
+    auto wait_warp = [&](uint32_t bar, uint32_t parity, volatile int *ab, WsHeader *h, uint32_t site) {
+      return __all_sync(0xffffffffu, wait_bar(bar, parity, ab, h, site));
+    };
+    {
       constexpr uint32_t idesc_s = make_idesc_f16(BF16, kDcRows, kDcKeys, false, false);
       constexpr uint32_t idesc_o = make_idesc_f16(BF16, kDcRows, 256, false, true);
-      const uint32_t s_tmem = tmem + (16u << 16);  // S chains and Q: lanes 16-31 of each sub-partition
+      const uint32_t tmem_w = __shfl_sync(0xffffffffu, tmem, 0);
+      const uint32_t s_tmem = tmem_w + (16u << 16);  // S chains and Q: lanes 16-31 of each sub-partition
       uint32_t tc = 0, g = 0, o_uses = 0;
       bool ok = true;
       // Descriptors: the high halves are fixed, a chunk / K-step only moves
@@ -317,38 +325,38 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       // S of tile counter `t` into the three chains (chunk c accumulates into chain c % 3).
       auto issue_s = [&](uint32_t t) -> bool {
         const int x = t % kDcRingTiles;
-        if (!wait_bar(b_tf(x), (t / kDcRingTiles) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
+        if (!wait_warp(b_tf(x), (t / kDcRingTiles) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
         tc_fence_after();
         const uint32_t k_lo = k_lo0 + (uint32_t)((x * kDcChunks * kDcChunkBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
           for (int c = 0; c < kDcChunks; ++c)
-            mma_ts2(s_tmem + (c % 3) * kDcKeys, s_tmem + kDcQCol + (c * 4 + kk) * 8,
+            if (leader) mma_ts2(s_tmem + (c % 3) * kDcKeys, s_tmem + kDcQCol + (c * 4 + kk) * 8,
                     k_lo + (uint32_t)((c * kDcChunkBytes + kk * 32) >> 4), k_hi, idesc_s, (c >= 3 || kk > 0) ? 1u : 0u);
-        mma_commit(b_sf);
+        if (leader) mma_commit(b_sf);
         return true;
       };
       for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
         const int4 sd = s.segs[sg];
         const int n = sd.z - sd.y;
-        if (!wait_bar(b_qr, (sg - seg_lo) & 1, abort_flag, hdr, kDSiteQReady)) break;
+        if (!wait_warp(b_qr, (sg - seg_lo) & 1, abort_flag, hdr, kDSiteQReady)) break;
         tc_fence_after();
-        if (g > 0 && !wait_bar(b_sx, (g - 1) & 1, abort_flag, hdr, kDSiteSFree)) break;
+        if (g > 0 && !wait_warp(b_sx, (g - 1) & 1, abort_flag, hdr, kDSiteSFree)) break;
         if (!issue_s(tc)) break;
         for (int jj = 0; jj < n; ++jj, ++g, ++tc) {
           if (jj + 1 < n) {
             // the single S buffer is free once softmax has read S(g)
-            if (!wait_bar(b_sx, g & 1, abort_flag, hdr, kDSiteSFree) || !issue_s(tc + 1)) {
+            if (!wait_warp(b_sx, g & 1, abort_flag, hdr, kDSiteSFree) || !issue_s(tc + 1)) {
               ok = false;
               break;
             }
           }
-          if (!wait_bar(b_pf, g & 1, abort_flag, hdr, kDSitePFull)) {
+          if (!wait_warp(b_pf, g & 1, abort_flag, hdr, kDSitePFull)) {
             ok = false;
             break;
           }
-          if (jj == 0 && o_uses > 0 && !wait_bar(b_oe, (o_uses - 1) & 1, abort_flag, hdr, kDSiteOEmpty)) {
+          if (jj == 0 && o_uses > 0 && !wait_warp(b_oe, (o_uses - 1) & 1, abort_flag, hdr, kDSiteOEmpty)) {
             ok = false;
             break;
           }
@@ -358,15 +366,15 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
           for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
             for (int half = 0; half < 2; ++half)
-              mma_ss2(tmem + half * 256, p_lo0 + (uint32_t)(kk * 2), p_hi,
+              if (leader) mma_ss2(tmem_w + half * 256, p_lo0 + (uint32_t)(kk * 2), p_hi,
                       v_lo + (uint32_t)((half * 4 * kDcChunkBytes + kk * 16 * 128) >> 4), v_hi, idesc_o,
                       (jj > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(b_od);
-          mma_commit(b_te(tc % kDcRingTiles));
+          if (leader) mma_commit(b_od);
+          if (leader) mma_commit(b_te(tc % kDcRingTiles));
         }
         ++o_uses;
       }
-      mma_commit(smem_u32(&ctrl->drain));
+      if (leader) mma_commit(smem_u32(&ctrl->drain));
       const uint64_t t0 = global_ns();
       while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < kWaitBudgetNs) {
       }

@@ -231,12 +231,6 @@ __device__ __forceinline__ float exp_store(const uint32_t (&sr)[N], int lim, flo
   return lo + hi;
 }
 
-// One lane of a converged warp (elect.sync).
-__device__ __forceinline__ bool elect_one() {
-  uint32_t r;
-  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(r));
-  return r != 0;
-}
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }

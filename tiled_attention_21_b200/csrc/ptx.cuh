@@ -312,6 +312,13 @@ __device__ __forceinline__ void regs_inc() {
 }
 
 // ---------------------------------------------------------------- math
+// One lane of a converged warp (elect.sync).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t r;
+  asm volatile("{\n .reg .pred p;\n elect.sync _|p, 0xffffffff;\n selp.u32 %0, 1, 0, p;\n}\n" : "=r"(r));
+  return r != 0;
+}
+
 // 2^x on the multi-function unit (ex2.approx: 2 ulp; 2^-inf = +0).
 __device__ __forceinline__ float ex2(float x) {
   float y;
