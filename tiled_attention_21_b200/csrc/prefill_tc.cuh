@@ -6,11 +6,11 @@
 // (128 keys) and query tile t:
 //     S_t  = Q_t K_j^T           tcgen05.mma, A = Q (smem), B = K (smem),
 //                                fp32 accumulator in TMEM
-//     P_t  = exp2(c*S_t - m)     softmax, two threads per row (one per
-//                                64-key half), c = softmax_scale*log2(e);
+//     P_t  = exp2(c*S_t - m)     softmax, four threads per row (one per
+//                                32-key group g), c = softmax_scale*log2(e);
 //                                P written back into TMEM over S_t as
-//                                bf16/f16 (keys 0-63 in columns 0-31,
-//                                keys 64-127 in columns 64-95)
+//                                bf16/f16 (keys 32g..32g+31 in columns
+//                                32g..32g+15)
 //     O_t += P_t V_j             tcgen05.mma, A = P (TMEM), B = V (smem)
 // The online-softmax bookkeeping follows mxflashattn 1.4.0 prefill.py
 // (prefill_chunked_reference: running max, correction of the accumulator,
@@ -23,16 +23,16 @@
 // Roles (640 threads, five warpgroups):
 //   warp 0      TMA producer: Q tiles once per unit, then K_j, V_j into a
 //               ring of shared-memory slots (128B-swizzled boxes of 64 cols)
-//   warp 1      TMEM allocator and single-thread MMA issuer; it alternates
-//               the two query tiles (PV_0(j), S_0(j+1), PV_1(j), S_1(j+1))
-//               so one tile's softmax overlaps the other tile's MMAs
-//   warps 4-11  softmax + epilogue of query tile 0, warps 12-19 of tile 1.
-//               A query row has two threads in two warps of the same TMEM
-//               sub-partition (warp w reads lanes 32*(w%4)..+31): one takes
-//               key columns 0-63 and output columns 0..D/2-1, the other the
-//               upper halves; they swap partial row maxima through shared
-//               memory (a 64-thread named barrier per pair of warps).
-// The first warpgroup gives registers to the softmax warpgroups (setmaxnreg).
+//   warp 1      TMEM allocator and MMA issuer: the whole warp runs the
+//               schedule and one elected lane issues; it alternates the two
+//               query tiles (PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)) so one
+//               tile's softmax overlaps the other tile's MMAs
+//   warps 4-19  softmax + epilogue.  A query row has four threads, one per
+//               32-key group g = (warp-4)/4, in the four warps of its TMEM
+//               sub-partition (warp w reads lanes 32*(w%4)..+31); these four
+//               warps take query tile 0 and query tile 1 in turn, and vote
+//               (bar.red.and) on whether the stale base still bounds every
+//               row before exchanging partial maxima through shared memory.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
 //
 // Every wait is bounded (see wait_bar); a wait that runs out records
