@@ -51,16 +51,17 @@ namespace mxfa {
 constexpr int kTcBlockM = 128;  // rows per query tile
 constexpr int kTcBlockN = 128;  // keys per KV tile
 constexpr int kTcUnitRows = 2 * kTcBlockM;
-constexpr int kTcThreads = 640;
-constexpr int kTcSoftmaxThreads = 512;  // four warpgroups: (query tile, column half)
-// Register budgets: launched at kTcLaunchRegs per thread; if the budgets of
-// the producer/MMA warpgroup (kTcRegsIo) and of the four softmax warpgroups
-// (kTcRegsSoftmax) differ, setmaxnreg moves registers between them, and
-// 128*kTcRegsIo + 512*kTcRegsSoftmax must not exceed 640*kTcLaunchRegs (the
-// host refuses to launch a build whose register count differs from
-// kTcLaunchRegs).  The softmax reads S in 32-column pieces so both fit in 96.
-constexpr int kTcLaunchRegs = 96, kTcRegsIo = 96, kTcRegsSoftmax = 96;
-static_assert(128 * kTcRegsIo + kTcSoftmaxThreads * kTcRegsSoftmax <= kTcThreads * kTcLaunchRegs, "register split");
+constexpr int kTcThreads = 768;
+constexpr int kTcSoftmaxThreads = 512;  // four warpgroups: four threads per query row
+constexpr int kTcEpiWarp0 = 20;         // warps 20-23: output epilogue
+// Register budgets: launched at kTcLaunchRegs per thread; setmaxnreg moves
+// registers from the producer/MMA warpgroup (kTcRegsIo) and the epilogue
+// warpgroup (kTcRegsEpi) to the four softmax warpgroups (kTcRegsSoftmax).
+// The split must fit in what the block was launched with (the host refuses
+// to launch a build whose register count differs from kTcLaunchRegs).
+constexpr int kTcLaunchRegs = 80, kTcRegsIo = 48, kTcRegsSoftmax = 96, kTcRegsEpi = 48;
+static_assert(128 * kTcRegsIo + kTcSoftmaxThreads * kTcRegsSoftmax + 128 * kTcRegsEpi <= kTcThreads * kTcLaunchRegs,
+              "register split");
 constexpr int kTcMaxSlots = 10;
 
 template <int D>
@@ -79,6 +80,7 @@ struct PrefillCtrl {
   uint64_t q_full, q_empty;
   uint64_t slot_full[kTcMaxSlots], slot_empty[kTcMaxSlots];
   uint64_t s_full[2], p_full[2], o_done[2], o_empty[2];
+  uint64_t l_ready, l_free;  // per unit: row sums handed to the epilogue warpgroup
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -88,7 +90,7 @@ struct PrefillCtrl {
 // Wait-site codes reported in the workspace on a timeout.
 enum : uint32_t {
   kSiteQEmpty = 0x101, kSiteSlotEmpty, kSiteQFull, kSiteSlotFull, kSitePFull, kSiteOEmpty,
-  kSiteSFull, kSiteODone, kSiteDrain
+  kSiteSFull, kSiteODone, kSiteDrain, kSiteLReady, kSiteLFree
 };
 
 struct UnitInfo {
@@ -289,9 +291,11 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       mbar_init(smem_u32(&ctrl->s_full[t]), 1);
       mbar_init(smem_u32(&ctrl->p_full[t]), kTcSoftmaxThreads / 32);  // one arrival per softmax warp
       mbar_init(smem_u32(&ctrl->o_done[t]), 1);
-      mbar_init(smem_u32(&ctrl->o_empty[t]), kTcSoftmaxThreads / 32);
+      mbar_init(smem_u32(&ctrl->o_empty[t]), 4);  // the epilogue warps
     }
     mbar_init(smem_u32(&ctrl->drain), 1);
+    mbar_init(smem_u32(&ctrl->l_ready), 4);  // softmax warps of column group 0
+    mbar_init(smem_u32(&ctrl->l_free), 4);   // the epilogue warps
     ctrl->abort = 0;
     fence_mbar_init();
   }
@@ -392,13 +396,13 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
                   k_lo + (uint32_t)((((kk >> 2) * Cfg::kAtomBytes) + (kk & 3) * 32) >> 4), sd_hi, idesc_s, kk > 0 ? 1u : 0u);
         if (leader) mma_commit(smem_u32(&ctrl->s_full[t]));
       };
-      auto issue_pv = [&](int t, int slot, bool acc) {
+      auto issue_pv = [&](int t, int slot, bool acc, bool last) {
         const uint32_t v_lo = vring_lo + (uint32_t)((slot * Cfg::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kTcBlockN / 16; ++kk)
           if (leader) mma_ts2(o_tm[t], s_tm[t] + (kk >> 1) * 32 + (kk & 1) * 8, v_lo + (uint32_t)(kk * 128), vd_hi, idesc_o,
                   (acc || kk > 0) ? 1u : 0u);
-        if (leader) mma_commit(smem_u32(&ctrl->o_done[t]));
+        if (leader && last) mma_commit(smem_u32(&ctrl->o_done[t]));  // O_t of the unit is complete
       };
       int it = 0;
       bool ok = true;
@@ -452,7 +456,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
               break;
             }
             tc_fence_after();
-            issue_pv(t, vs, j > 0);
+            issue_pv(t, vs, j > 0, j + 1 == ui.n[t]);
             if (j + 1 < ui.n[t]) {
               if (!kwaited) {
                 if (!wait_warp(b_sf(ks), kph, abort_flag, hdr, kSiteSlotFull)) {
@@ -481,7 +485,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       }
     }
   }
-  } else {
+  } else if (warp < kTcEpiWarp0) {
     if constexpr (kTcRegsSoftmax != kTcLaunchRegs) regs_inc<kTcRegsSoftmax>();
     // ------------------------------------------------------------ softmax / epilogue
     // Four threads per query row, one per 32-key column group g; the four
@@ -504,6 +508,14 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       const int nmax = max(ui.n[0], ui.n[1]);
       int i[2], nv[2];
       float m_used[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      {
+        // the exchange area holds the previous unit's row sums until the
+        // epilogue warpgroup has taken them
+        bool lf = true;
+        if (it > 0) lf = wait_bar(smem_u32(&ctrl->l_free), (it - 1) & 1, abort_flag, hdr, kSiteLFree);
+        __syncwarp();
+        if (bar_or(bar_id, 128, !__all_sync(0xffffffffu, lf))) break;
+      }
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         i[t] = ui.m * kTcUnitRows + t * kTcBlockM + r;
@@ -585,53 +597,89 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         }
       }
       if (!ok) break;
-      // epilogue of both query tiles
+      // Row sums over the four groups and the LSE; the sums go to the
+      // epilogue warpgroup through the exchange area (xchg[t][row]).
+      float lt[2];
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        bool got_o = true;
-        if (ui.n[t] > 0) got_o = wait_bar(smem_u32(&ctrl->o_done[t]), (pv_cnt[t] - 1) & 1, abort_flag, hdr, kSiteODone);
-        __syncwarp();
-        if (bar_or(bar_id, 128, !__all_sync(0xffffffffu, got_o))) {
-          ok = false;
-          break;
-        }
-        // row sum over the four groups
         *x_mine = l[t];
         named_bar_sync(bar_id, 128);
-        const float lt = (ctrl->xchg[0][r] + ctrl->xchg[1][r]) + (ctrl->xchg[2][r] + ctrl->xchg[3][r]);
-        named_bar_sync(bar_id, 128);
-        const bool valid = i[t] < ui.sr.sq;
-        using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-        T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(ui.sr.q0 + i[t]) * p.o_rs + (int64_t)ui.h * p.o_hs + g * OC;
+        lt[t] = (ctrl->xchg[0][r] + ctrl->xchg[1][r]) + (ctrl->xchg[2][r] + ctrl->xchg[3][r]);
+        named_bar_sync(bar_id, 128);  // all have read before the hand-over is written
+        if (i[t] < ui.sr.sq && g == 0 && p.lse)
+          p.lse[(int64_t)(ui.sr.q0 + i[t]) * p.hq + ui.h] =
+              lt[t] > 0.f ? (m_used[t] + __log2f(lt[t])) * 0.69314718055994530942f : -INFINITY;
+      }
+      if (g == 0) {
+        ctrl->xchg[0][r] = lt[0];
+        ctrl->xchg[1][r] = lt[1];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ctrl->l_ready));
+      }
+    }
+  } else {
+    if constexpr (kTcRegsEpi != kTcLaunchRegs) regs_dec<kTcRegsEpi>();
+    // ------------------------------------------------------------ output epilogue
+    // Warps 20-23, one thread per query row (warp w reads TMEM lanes
+    // 32*(w%4)..+31): O_t / l in the output dtype once the unit's last P.V of
+    // tile t is complete; then O_t's TMEM columns are released to the MMAs.
+    const int sub = warp & 3;
+    const int r = sub * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16);
+    const bool o_v8 = ((reinterpret_cast<uintptr_t>(p.o) | (uintptr_t)(p.o_rs * 2) | (uintptr_t)(p.o_hs * 2)) & 31u) == 0;
+    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    uint32_t o_cnt[2] = {0, 0};
+    bool ok = true;
+    for (int it = 0, u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
+      const UnitInfo ui = unit_info(p, u);
+      const bool got_l = wait_bar(smem_u32(&ctrl->l_ready), it & 1, abort_flag, hdr, kSiteLReady);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got_l)) break;
+      const float lt0 = ctrl->xchg[0][r], lt1 = ctrl->xchg[1][r];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctrl->l_free));
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float lt = t ? lt1 : lt0;
+        const int i = ui.m * kTcUnitRows + t * kTcBlockM + r;
+        const bool valid = i < ui.sr.sq;
+        T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(ui.sr.q0 + i) * p.o_rs + (int64_t)ui.h * p.o_hs;
         if (ui.n[t] > 0) {
+          const bool got_o = wait_bar(smem_u32(&ctrl->o_done[t]), o_cnt[t] & 1, abort_flag, hdr, kSiteODone);
+          __syncwarp();
+          if (!__all_sync(0xffffffffu, got_o)) {
+            ok = false;
+            break;
+          }
+          ++o_cnt[t];
           tc_fence_after();
           const float inv = lt > 0.f ? 1.f / lt : 0.f;
-          const uint32_t oa = trow + 2 * kTcBlockN + t * D + g * OC;
-          uint32_t ov[OC];
-          if constexpr (OC == 32) tmem_ld32(oa, ov);
-          else tmem_ld16(oa, ov);
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t ov[16], pk[8];
+            tmem_ld16(trow + 2 * kTcBlockN + t * D + c * 16, ov);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float a0 = __uint_as_float(ov[2 * e]) * inv, a1 = __uint_as_float(ov[2 * e + 1]) * inv;
+              pk[e] = BF16 ? pack_bf16x2(a0, a1) : pack_f16x2(a0, a1);
+            }
+            if (valid) {
+              if (o_v8) {
+                st_global_v8(orow + c * 16, pk);
+              } else {
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 16);
+                dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+              }
+            }
+          }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&ctrl->o_empty[t]));
-          uint32_t pk[OC / 2];
-#pragma unroll
-          for (int e = 0; e < OC / 2; ++e) {
-            const float a0 = __uint_as_float(ov[2 * e]) * inv, a1 = __uint_as_float(ov[2 * e + 1]) * inv;
-            pk[e] = BF16 ? pack_bf16x2(a0, a1) : pack_f16x2(a0, a1);
-          }
-          if (valid) {
-            uint4 *dst = reinterpret_cast<uint4 *>(orow);
-#pragma unroll
-            for (int e = 0; e < OC / 8; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-          }
         } else if (valid) {
           uint4 *dst = reinterpret_cast<uint4 *>(orow);
 #pragma unroll
-          for (int e = 0; e < OC / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
-        }
-        if (valid && g == 0 && p.lse) {
-          p.lse[(int64_t)(ui.sr.q0 + i[t]) * p.hq + ui.h] =
-              lt > 0.f ? (m_used[t] + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+          for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
         }
       }
     }

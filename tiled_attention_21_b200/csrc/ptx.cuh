@@ -319,6 +319,13 @@ __device__ __forceinline__ bool elect_one() {
   return r != 0;
 }
 
+// 32-byte global store (one 256-bit access); the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void *ptr, const uint32_t *v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 // 2^x on the multi-function unit (ex2.approx: 2 ulp; 2^-inf = +0).
 __device__ __forceinline__ float ex2(float x) {
   float y;
