@@ -325,7 +325,7 @@ def main():
         dd = to_dev(pdc, dev)
         od = torch.empty((pdc.total_q, pdc.hq, pdc.dv), dtype=torch.bfloat16, device=dev)
         ld = torch.empty((pdc.total_q, pdc.hq), dtype=torch.float32, device=dev)
-        need = mx.load().mxfa_attn_decode_splitkv_workspace_size(pdc.batch, 4, pdc.hq, pdc.dv, 8192, 0, 2)
+        need = mx.load().mxfa_attn_decode_splitkv_workspace_size(pdc.batch, 4, pdc.hq, 1, pdc.dv, 8192, 0, 2)
         wsd = torch.zeros(need + 256, dtype=torch.uint8, device=dev)
 
         def dstep():

@@ -152,13 +152,19 @@ mxfa_status_t mxfa_attn_varlen_fwd_noalloc(const void *q, const void *k, const v
  * Dqk = 576, Dv = 512, k_row_stride = v_row_stride = 576: value = first 512
  * columns of each cached row; the tensor-core kernel reads each KV tile once
  * and uses it as both operands.  That path needs bf16/f16 and
- * max_q_len * Hq <= 64.  Other shapes ((Dqk, Dv) = (64, 64) or (128, 128),
- * or f32) run on the exact CUDA-core kernel.
+ * max_q_len * Hq <= 64.
+ * Grouped-query decode (mxflashattn flash_attn_with_kvcache shape): Dqk = Dv
+ * = 64 or 128, bf16/f16, max_q_len * (Hq / Hkv) <= 64 and row strides that
+ * are multiples of 8 elements run on the tensor-core kernel, which streams
+ * each KV head once for the Hq / Hkv query heads that share it.  Other shapes
+ * (or f32) run on the exact CUDA-core kernel.
+ * The workspace size takes Hkv because the grouped-query kernel schedules
+ * batch * Hkv decode sequences.
  * num_splits: 0 = automatic (the KV of all sequences is cut into
  *   near-equal pieces, one run per SM); k >= 1 = every sequence's KV is cut
  *   into k pieces.  The result does not depend on it beyond fp32 rounding.
  */
-size_t mxfa_attn_decode_splitkv_workspace_size(int batch, int max_q_len, int Hq, int Dv, int max_kv_len,
+size_t mxfa_attn_decode_splitkv_workspace_size(int batch, int max_q_len, int Hq, int Hkv, int Dv, int max_kv_len,
                                                int num_splits, mxfa_dtype_t dtype);
 mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
                                        const int32_t *qo_indptr, const int32_t *kv_indptr,

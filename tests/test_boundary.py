@@ -102,6 +102,12 @@ def test_workspace_sizes(lib):
     big = lib.mxfa_attn_varlen_fwd_workspace_size(64, 32768, 32768, 8, 128, 2)
     assert 256 < small < big
     assert lib.mxfa_attn_varlen_fwd_workspace_size(2, 128, 128, 8, 128, 0) == 256  # fp32 path needs no schedule
+    mla = lib.mxfa_attn_decode_splitkv_workspace_size(128, 4, 16, 1, 512, 8192, 0, 2)
+    gqa = lib.mxfa_attn_decode_splitkv_workspace_size(64, 1, 32, 4, 128, 8192, 0, 2)
+    assert mla > 256 and gqa > 256
+    # the grouped-query schedule covers batch * Hkv sequences
+    assert lib.mxfa_attn_decode_splitkv_workspace_size(64, 1, 32, 8, 128, 8192, 0, 2) > gqa
+    assert lib.mxfa_attn_decode_splitkv_workspace_size(64, 1, 32, 4, 128, 8192, 0, 0) == 256  # fp32
 
 
 def test_product_path_does_not_touch_the_oracle():

@@ -20,7 +20,7 @@ def _lib():
 
 def check(p, num_splits=0, pairs=None):
     d = to_dev(p)
-    o, l = run(p, d, num_splits=num_splits)
+    o, l = run(p, d, "decode", num_splits=num_splits)
     torch.cuda.synchronize()
     if pairs is None:
         ro, rl = oracle.problem(p)
@@ -67,4 +67,57 @@ def test_gqa_decode(dims, dt):
 def test_full_size_mla_sampled():
     p = workloads.cfg_mla_decode()
     pairs = workloads.sample_rows(p, 16, 104)
+    check(p, 0, pairs)
+
+
+# ---------------------------------------------------------------- grouped-query decode on the tensor cores
+@pytest.mark.parametrize("splits", [0, 1, 3, 8])
+def test_gqa_tc_small(splits):
+    p = workloads.gqa_decode(31, batch=3, q_len=1, kv_len=700)
+    check(p, splits)
+
+
+def test_gqa_tc_ragged_and_empty_lengths():
+    # a sequence without keys ends at O = 0, LSE = -inf (written by the combine pass)
+    p = workloads.gqa_decode(32, batch=6, q_len=1, kv_len=0, lens_kv=[1, 64, 65, 1000, 0, 129])
+    check(p)
+    check(p, 2)
+
+
+@pytest.mark.parametrize("q_len,causal", [(4, True), (4, False), (8, True)])
+def test_gqa_tc_several_queries(q_len, causal):
+    # q_len * G rows per KV head: 32, 32 and 64 (the largest the kernel takes)
+    p = workloads.gqa_decode(33, batch=3, q_len=q_len, kv_len=333, causal=causal)
+    check(p)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_gqa_tc_d64(dt):
+    p = workloads.gqa_decode(34, batch=4, q_len=2, kv_len=517, hq=16, hkv=2, d=64, dtype=dt)
+    check(p)
+    check(p, 3)
+
+
+def test_gqa_tc_group_sizes():
+    # G = 1 (one query head per KV head) and G = 16
+    check(workloads.gqa_decode(35, batch=2, q_len=1, kv_len=300, hq=8, hkv=8))
+    check(workloads.gqa_decode(36, batch=2, q_len=2, kv_len=300, hq=32, hkv=2))
+
+
+def test_gqa_rows_beyond_tensor_core_limit():
+    # q_len * G = 128 > 64 rows: the exact CUDA-core kernel takes it
+    check(workloads.gqa_decode(37, batch=2, q_len=16, kv_len=200, causal=True))
+
+
+def test_gqa_tc_split_invariance():
+    p = workloads.gqa_decode(38, batch=2, q_len=1, kv_len=4096)
+    _, (o1, l1) = check(p, 1)
+    _, (o8, l8) = check(p, 8)
+    assert (o1.float() - o8.float()).abs().max() <= 4e-3
+    assert (l1 - l8).abs().max() <= 1e-4
+
+
+def test_full_size_gqa_sampled():
+    p = workloads.cfg_gqa_decode()
+    pairs = workloads.sample_rows(p, 16, 105)
     check(p, 0, pairs)

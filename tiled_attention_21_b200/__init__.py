@@ -54,7 +54,7 @@ def load():
             lib.mxfa_attn_varlen_fwd_workspace_size.restype = sz
             lib.mxfa_attn_decode_splitkv.argtypes = [vp] * 7 + [i32] * 9 + [i64, i64, i32, f32, i32, i32, vp, sz, vp]
             lib.mxfa_attn_decode_splitkv.restype = i32
-            lib.mxfa_attn_decode_splitkv_workspace_size.argtypes = [i32] * 7
+            lib.mxfa_attn_decode_splitkv_workspace_size.argtypes = [i32] * 8
             lib.mxfa_attn_decode_splitkv_workspace_size.restype = sz
             lib.mxfa_last_error.argtypes = []
             lib.mxfa_last_error.restype = ctypes.c_char_p
@@ -193,7 +193,7 @@ def mxfa_attn_decode_splitkv(q, k, v, qo_indptr, kv_indptr, max_q_len: int, max_
     if lse is None and return_lse:
         lse = torch.empty((total_q, Hq), dtype=torch.float32, device=q.device)
     dt = _DT[q.dtype]
-    need = lib.mxfa_attn_decode_splitkv_workspace_size(batch, max_q_len, Hq, Dv, max_kv_len, num_splits, dt)
+    need = lib.mxfa_attn_decode_splitkv_workspace_size(batch, max_q_len, Hq, Hkv, Dv, max_kv_len, num_splits, dt)
     ws = ws if ws is not None else workspace(need, q.device)
     wp, wn = _ws_view(ws)
     _check(lib.mxfa_attn_decode_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(qo_indptr),

@@ -56,13 +56,17 @@ constexpr int kDcSmemBytes = kDcCtrlBytes + kDcSlots * kDcChunkBytes + kDcRows *
 static_assert(kDcSmemBytes <= 232448, "shared memory budget");
 constexpr int kDcMaxGrid = 256;
 
+// A decode "sequence" v is (batch entry b, KV head g) = (v / heads, v % heads):
+// heads = 1 for MLA (all query heads share the one latent KV head), Hkv for
+// grouped-query decode (the G = Hq/Hkv query heads of KV head g).
 struct DecodeSched {
-  int *n_tiles;    // [batch] KV tiles per sequence
-  int *tile_pre;   // [batch + 1] prefix of n_tiles
-  int *seg_base;   // [batch + 1] first segment of each sequence
-  int *seg_cnt;    // [batch]
-  int4 *segs;      // [max_segs] (b, first tile, end tile, global first tile)
-  float *part_acc; // [max_segs][64][512]
+  int heads;       // KV heads per batch entry that form separate sequences
+  int *n_tiles;    // [batch*heads] KV tiles per sequence
+  int *tile_pre;   // [batch*heads + 1] prefix of n_tiles
+  int *seg_base;   // [batch*heads + 1] first segment of each sequence
+  int *seg_cnt;    // [batch*heads]
+  int4 *segs;      // [max_segs] (v, first tile, end tile, global first tile)
+  float *part_acc; // [max_segs][64][Dv]
   float2 *part_ml; // [max_segs][64] (running max in log2 units, running sum)
   int max_segs;
   int num_splits;  // 0 = automatic
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
   __shared__ typename Scan::TempStorage tmp;
   __shared__ int carry, max_n, split_mode;
   __shared__ int cut[kDcMaxGrid + 1];  // x_c = c*T/G, c = 0..G
-  const int tid = threadIdx.x, B = p.batch, G = s.grid;
+  const int tid = threadIdx.x, B = p.batch * s.heads, G = s.grid;
   if (tid == 0) {
     carry = 0;
     max_n = 0;
@@ -119,8 +123,9 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     const int b = base + tid;
     int n = 0;
     if (b < B) {
-      n = (p.cu_k[b + 1] - p.cu_k[b] + kDcKeys - 1) / kDcKeys;
-      if (p.cu_q[b + 1] - p.cu_q[b] <= 0) n = 0;  // no queries: nothing to compute
+      const int e = b / s.heads;  // batch entry of sequence b
+      n = (p.cu_k[e + 1] - p.cu_k[e] + kDcKeys - 1) / kDcKeys;
+      if (p.cu_q[e + 1] - p.cu_q[e] <= 0) n = 0;  // no queries: nothing to compute
       s.n_tiles[b] = n;
       atomicMax(&max_n, n);
     }
@@ -576,17 +581,20 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
 }
 
 // ----------------------------------------------------------------------------
-// Merge the pieces of every sequence that was split: block (row r, sequence b).
-template <typename T>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const AttnParams p, const DecodeSched s) {
-  const int r = blockIdx.x, b = blockIdx.y;
+// Merge the pieces of every sequence that was split: block (row r, sequence
+// v), DV/4 threads.  Row r of sequence v = (b, g) is query token r / G of
+// batch entry b, head g*G + r % G, with G = Hq / heads.
+template <typename T, int DV>
+__global__ void __launch_bounds__(DV / 4) decode_combine_kernel(const AttnParams p, const DecodeSched s) {
+  const int r = blockIdx.x, v = blockIdx.y;
+  const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
   const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
-  if (r >= sq * p.hq) return;
-  const int cnt = s.seg_cnt[b];
+  if (r >= sq * G) return;
+  const int cnt = s.seg_cnt[v];
   if (cnt == 1) return;  // stored directly by the decode kernel
-  const int tok = q0 + r / p.hq, h = r % p.hq;
+  const int tok = q0 + r / G, h = gh * G + r % G;
   T *orow = reinterpret_cast<T *>(p.o) + (int64_t)tok * p.o_rs + (int64_t)h * p.o_hs;
-  const int base = s.seg_base[b];
+  const int base = s.seg_base[v];
   float M = -INFINITY;
   for (int i = 0; i < cnt; ++i) M = fmaxf(M, s.part_ml[(int64_t)(base + i) * kDcRows + r].x);
   float L = 0.f;
@@ -596,7 +604,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const AttnParams p,
       const float2 ml = s.part_ml[(int64_t)(base + i) * kDcRows + r];
       const float w = ex2(ml.x - M);  // 0 for a piece that saw no visible key
       L += w * ml.y;
-      const float4 a = reinterpret_cast<const float4 *>(s.part_acc + ((int64_t)(base + i) * kDcRows + r) * kDcDv)[threadIdx.x];
+      const float4 a = reinterpret_cast<const float4 *>(s.part_acc + ((int64_t)(base + i) * kDcRows + r) * DV)[threadIdx.x];
       acc[0] = fmaf(w, a.x, acc[0]);
       acc[1] = fmaf(w, a.y, acc[1]);
       acc[2] = fmaf(w, a.z, acc[2]);

@@ -27,6 +27,7 @@
 #include "prefill_tc.cuh"
 #include "sched.cuh"
 #include "decode_tc.cuh"
+#include "decode_gqa.cuh"
 
 using namespace mxfa;
 
@@ -134,16 +135,16 @@ mxfa_status_t get_encoder(EncodeTiledFn *fn) {
   return MXFA_OK;
 }
 
-// 3-D map over [rows][heads][D] (16-bit elements), box = 128 rows x 1 head x
-// 64 columns, 128-byte swizzle; rows past `rows` read as zero.
+// 3-D map over [rows][heads][D] (16-bit elements), box = `box_rows` rows x
+// 1 head x 64 columns, 128-byte swizzle; rows past `rows` read as zero.
 mxfa_status_t make_map(CUtensorMap *map, const void *base, mxfa_dtype_t dt, int D, int heads, int64_t rows,
-                       int64_t row_stride, int64_t head_stride) {
+                       int64_t row_stride, int64_t head_stride, int box_rows = kTcBlockM) {
   EncodeTiledFn enc;
   mxfa_status_t st = get_encoder(&enc);
   if (st != MXFA_OK) return st;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)(rows > 0 ? rows : 1)};
   cuuint64_t strides[2] = {(cuuint64_t)head_stride * 2, (cuuint64_t)row_stride * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTcBlockM};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, dt == MXFA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -302,12 +303,14 @@ mxfa_status_t prefill(AttnParams &p, mxfa_dtype_t dt, int D, bool varlen, int64_
   return bf ? launch_tc<64, true>(p, mq, mk, mv, st) : launch_tc<64, false>(p, mq, mk, mv, st);
 }
 
-// Workspace layout of the tensor-core MLA decode.
+// Workspace layout of the tensor-core decode kernels: `batch` decode
+// sequences (batch entries x KV heads that form separate sequences), Dv
+// output columns.
 struct DecodeWs {
   size_t n_tiles, tile_pre, seg_base, seg_cnt, segs, part_ml, part_acc, total;
   int max_segs;
 };
-DecodeWs decode_ws(int batch, int max_kv_len, int num_splits) {
+DecodeWs decode_ws(int batch, int max_kv_len, int num_splits, int dv) {
   DecodeWs w;
   const int tiles = (max_kv_len + kDcKeys - 1) / kDcKeys;
   w.max_segs = num_splits > 0 ? batch * std::max(1, std::min(num_splits, tiles)) : batch + kDcMaxGrid;
@@ -318,7 +321,7 @@ DecodeWs decode_ws(int batch, int max_kv_len, int num_splits) {
   w.segs = w.seg_cnt + align256(sizeof(int) * (size_t)batch);
   w.part_ml = w.segs + align256(sizeof(int4) * (size_t)w.max_segs);
   w.part_acc = w.part_ml + align256(sizeof(float2) * (size_t)w.max_segs * kDcRows);
-  w.total = w.part_acc + align256(sizeof(float) * (size_t)w.max_segs * kDcRows * kDcDv);
+  w.total = w.part_acc + align256(sizeof(float) * (size_t)w.max_segs * kDcRows * dv);
   return w;
 }
 
@@ -328,13 +331,20 @@ bool decode_tc_eligible(mxfa_dtype_t dt, int Hq, int Hkv, int Dqk, int Dv, int m
          (int64_t)max_q_len * Hq <= kDcRows;
 }
 
-mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int total_kv, int num_splits, void *ws,
-                               cudaStream_t st) {
-  int sms = 0;
-  MXFA_TRY(sm_count(&sms));
-  const DecodeWs w = decode_ws(p.batch, p.max_sk, num_splits);
+// The grouped-query tensor-core decode: K and V heads of dimension 64 or 128,
+// 16-bit, q_len x G <= 64 query rows per KV head, rows TMA-addressable.
+bool decode_gqa_eligible(mxfa_dtype_t dt, int Hq, int Hkv, int Dqk, int Dv, int max_q_len, int64_t k_rs,
+                         int64_t v_rs) {
+  return dt != MXFA_F32 && Dqk == Dv && (Dqk == 64 || Dqk == 128) && (int64_t)max_q_len * (Hq / Hkv) <= kDcRows &&
+         (k_rs * 2) % 16 == 0 && (v_rs * 2) % 16 == 0;
+}
+
+// Split schedule in the workspace for `heads` decode sequences per batch entry.
+DecodeSched decode_sched(const AttnParams &p, int heads, int num_splits, int dv, void *ws, int sms) {
+  const DecodeWs w = decode_ws(p.batch * heads, p.max_sk, num_splits, dv);
   char *base = static_cast<char *>(ws);
   DecodeSched s;
+  s.heads = heads;
   s.n_tiles = reinterpret_cast<int *>(base + w.n_tiles);
   s.tile_pre = reinterpret_cast<int *>(base + w.tile_pre);
   s.seg_base = reinterpret_cast<int *>(base + w.seg_base);
@@ -345,6 +355,45 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
   s.max_segs = w.max_segs;
   s.num_splits = num_splits;
   s.grid = std::min(sms, kDcMaxGrid);
+  return s;
+}
+
+template <int D, bool BF16>
+mxfa_status_t launch_decode_gqa_t(AttnParams &p, mxfa_dtype_t dt, int total_kv, int num_splits, void *ws,
+                                  cudaStream_t st) {
+  int sms = 0;
+  MXFA_TRY(sm_count(&sms));
+  const DecodeSched s = decode_sched(p, p.hkv, num_splits, D, ws, sms);
+  CUtensorMap mk, mv;
+  MXFA_TRY(make_map(&mk, p.k, dt, D, p.hkv, total_kv, p.k_rs, p.k_hs, kDcKeys));
+  MXFA_TRY(make_map(&mv, p.v, dt, D, p.hkv, total_kv, p.v_rs, p.v_hs, kDcKeys));
+  decode_prep_kernel<<<1, 1024, 0, st>>>(p, s);
+  MXFA_CUDA(cudaGetLastError());
+  auto k = attn_decode_gqa_kernel<D, BF16>;
+  MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(k), GqaCfg<D>::kSmemBytes));
+  k<<<s.grid, kGqThreads, GqaCfg<D>::kSmemBytes, st>>>(p, s, mk, mv);
+  MXFA_CUDA(cudaGetLastError());
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  decode_combine_kernel<T, D><<<dim3(kDcRows, p.batch * p.hkv), D / 4, 0, st>>>(p, s);
+  MXFA_CUDA(cudaGetLastError());
+  return MXFA_OK;
+}
+
+mxfa_status_t launch_decode_gqa(AttnParams &p, mxfa_dtype_t dt, int total_kv, int num_splits, void *ws,
+                                cudaStream_t st) {
+  const bool bf = dt == MXFA_BF16;
+  if (p.dqk == 128)
+    return bf ? launch_decode_gqa_t<128, true>(p, dt, total_kv, num_splits, ws, st)
+              : launch_decode_gqa_t<128, false>(p, dt, total_kv, num_splits, ws, st);
+  return bf ? launch_decode_gqa_t<64, true>(p, dt, total_kv, num_splits, ws, st)
+            : launch_decode_gqa_t<64, false>(p, dt, total_kv, num_splits, ws, st);
+}
+
+mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int total_kv, int num_splits, void *ws,
+                               cudaStream_t st) {
+  int sms = 0;
+  MXFA_TRY(sm_count(&sms));
+  const DecodeSched s = decode_sched(p, 1, num_splits, kDcDv, ws, sms);
   CUtensorMap mq, mkv;
   MXFA_TRY(make_map_2d(&mq, p.q, dt, kDcDqk, (int64_t)total_q * p.hq, kDcDqk));
   MXFA_TRY(make_map_2d(&mkv, p.k, dt, kDcDqk, total_kv, p.k_rs));
@@ -354,12 +403,12 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
     MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(attn_decode_tc_kernel<true>), kDcSmemBytes));
     attn_decode_tc_kernel<true><<<s.grid, kDcThreads, kDcSmemBytes, st>>>(p, s, mq, mkv);
     MXFA_CUDA(cudaGetLastError());
-    decode_combine_kernel<__nv_bfloat16><<<dim3(kDcRows, p.batch), 128, 0, st>>>(p, s);
+    decode_combine_kernel<__nv_bfloat16, kDcDv><<<dim3(kDcRows, p.batch), kDcDv / 4, 0, st>>>(p, s);
   } else {
     MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(attn_decode_tc_kernel<false>), kDcSmemBytes));
     attn_decode_tc_kernel<false><<<s.grid, kDcThreads, kDcSmemBytes, st>>>(p, s, mq, mkv);
     MXFA_CUDA(cudaGetLastError());
-    decode_combine_kernel<__half><<<dim3(kDcRows, p.batch), 128, 0, st>>>(p, s);
+    decode_combine_kernel<__half, kDcDv><<<dim3(kDcRows, p.batch), kDcDv / 4, 0, st>>>(p, s);
   }
   MXFA_CUDA(cudaGetLastError());
   return MXFA_OK;
@@ -492,11 +541,14 @@ mxfa_status_t mxfa_attn_varlen_fwd(const void *q, const void *k, const void *v, 
   return prefill(p, dtype, D, true, total_q, total_k, workspace, st);
 }
 
-size_t mxfa_attn_decode_splitkv_workspace_size(int batch, int max_q_len, int Hq, int Dv, int max_kv_len,
+size_t mxfa_attn_decode_splitkv_workspace_size(int batch, int max_q_len, int Hq, int Hkv, int Dv, int max_kv_len,
                                                int num_splits, mxfa_dtype_t dtype) {
-  if (dtype == MXFA_F32 || Dv != kDcDv || batch <= 0 || (int64_t)max_q_len * Hq > kDcRows || num_splits < 0)
-    return sizeof(WsHeader);
-  return decode_ws(batch, max_kv_len, num_splits).total;
+  if (dtype == MXFA_F32 || batch <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || num_splits < 0) return sizeof(WsHeader);
+  if (Dv == kDcDv && Hkv == 1 && (int64_t)max_q_len * Hq <= kDcRows)  // MLA
+    return decode_ws(batch, max_kv_len, num_splits, kDcDv).total;
+  if ((Dv == 64 || Dv == 128) && (int64_t)max_q_len * (Hq / Hkv) <= kDcRows)  // grouped-query heads
+    return decode_ws(batch * Hkv, max_kv_len, num_splits, Dv).total;
+  return sizeof(WsHeader);
 }
 
 mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -529,8 +581,8 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
       return fail(MXFA_ERR_INVALID_ARG, "row strides smaller than a row");
   }
   MXFA_TRY(check_workspace(workspace, workspace_bytes,
-                           mxfa_attn_decode_splitkv_workspace_size(batch, max_q_len, Hq, Dv, max_kv_len, num_splits,
-                                                                   dtype)));
+                           mxfa_attn_decode_splitkv_workspace_size(batch, max_q_len, Hq, Hkv, Dv, max_kv_len,
+                                                                   num_splits, dtype)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (strict_mode()) {
     MXFA_TRY(strict_check_cu(qo_indptr, batch, total_q, max_q_len, "qo_indptr", st));
@@ -549,6 +601,8 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
   p.pairs = nullptr;
   if (decode_tc_eligible(dtype, Hq, Hkv, Dqk, Dv, max_q_len, k, v, k_row_stride, v_row_stride) && total_kv > 0)
     return launch_decode_tc(p, dtype, total_q, total_kv, num_splits, workspace, st);
+  if (decode_gqa_eligible(dtype, Hq, Hkv, Dqk, Dv, max_q_len, k_row_stride, v_row_stride) && total_kv > 0)
+    return launch_decode_gqa(p, dtype, total_kv, num_splits, workspace, st);
   return launch_simt_any(dtype, p, max_q_len, st);
 }
 

@@ -129,6 +129,17 @@ def mla_decode(seed: int, batch: int, q_len: int, kv_len: int, heads: int = 16, 
                    meta={"batch": batch, "q_len": q_len, "kv_len": kv_len})
 
 
+def gqa_decode(seed: int, batch: int, q_len: int, kv_len: int, hq: int = 32, hkv: int = 4, d: int = 128,
+               dtype: str = "bf16", causal: bool = False, lens_kv: list[int] | None = None,
+               name: str | None = None) -> Problem:
+    """Grouped-query decode on a dense KV cache: q [batch*q_len, hq, d], k/v
+    [total_kv, hkv, d] (the q_len = 1 decode bench shapes of AstrAI
+    attn_decode_split_kv_mma.cuh: Hq = 32, Hk = 4, D = 128)."""
+    lens_kv = [kv_len] * batch if lens_kv is None else lens_kv
+    return varlen(seed, [q_len] * batch, lens_kv, hq, hkv, d, dtype, causal,
+                  name=name or f"gqa_decode_b{batch}_q{q_len}_kv{kv_len}_hq{hq}_hkv{hkv}_d{d}_{dtype}")
+
+
 # ---------------------------------------------------------------------------
 # The five named workloads.
 # ---------------------------------------------------------------------------
@@ -168,6 +179,12 @@ def cfg_varlen_gqa() -> Problem:
 def cfg_mla_decode() -> Problem:
     """MLA split-KV decode, bf16: batch 128, q_len 4, 16 heads, 576/512, kv_len 8192; seed 3."""
     return mla_decode(3, 128, 4, 8192, name="mla_decode_b128_q4_h16_kv8192_bf16")
+
+
+def cfg_gqa_decode(batch: int = 64, kv_len: int = 8192) -> Problem:
+    """Grouped-query decode (next scope row): q_len 1, Hq 32, Hkv 4, D 128,
+    bf16, kv_len 8192 per sequence, seed 6; KV 1.07 GB, larger than L2."""
+    return gqa_decode(6, batch, 1, kv_len)
 
 
 def cfg_long_causal(S: int = 32768, H: int = 32, rows_per_head: int = 256) -> Problem:
