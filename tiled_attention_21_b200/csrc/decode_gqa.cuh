@@ -10,15 +10,15 @@
 // form the M = 64 side of every MMA (rows past q_len*G are zero and never
 // stored).
 //
-// The K and V heads of each sequence are streamed exactly once: 64-key tiles
-// arrive by TMA as D/64 column chunks of K followed by D/64 chunks of V
-// (64 keys x 64 columns, 128B swizzle) into a ring of kRingTiles tiles.
-//     S   = Q K^T   tcgen05.mma M=64 N=64, D/16 K-steps, A = Q (TMEM), B = K;
+// The K and V heads of each sequence are streamed exactly once: 128-key
+// tiles arrive by TMA as D/64 column chunks of K followed by D/64 chunks of
+// V (128 keys x 64 columns, 128B swizzle) into a ring of kRingTiles tiles.
+//     S   = Q K^T   tcgen05.mma M=64 N=128, D/16 K-steps, A = Q (TMEM), B = K;
 //                   the K-steps alternate between two accumulators so
 //                   consecutive MMAs do not wait on each other; softmax adds them
-//     O  += P V     tcgen05.mma M=64 N=D, A = P (shared memory), B = V
+//     O  += P V     tcgen05.mma M=64 N=D, 8 K-steps, A = P (shared memory), B = V
 // TMEM: O in lanes 0-15 of each sub-partition (columns 0..D-1); in lanes
-// 16-31 the two S accumulators (columns 0-127) and Q (columns 128..128+D/2).
+// 16-31 the two S accumulators (columns 0-255) and Q (columns 256..256+D/2).
 // Softmax, the lazy rescale of O, the epilogue, the partials of split
 // sequences and the bounded waits are those of the MLA kernel in
 // decode_tc.cuh; decode_combine_kernel merges the partials.
@@ -29,15 +29,18 @@
 namespace mxfa {
 
 constexpr int kGqThreads = 256;
-constexpr int kGqQCol = 128;  // first TMEM column of Q (lanes 16-31)
+constexpr int kGqKeys = 128;                    // keys per KV tile
+constexpr int kGqChunkBytes = kGqKeys * 128;    // one 64-column chunk of a tile
+constexpr int kGqPBytes = kDcRows * kGqKeys * 2;  // P: two 64-key blocks of 64 rows x 128 B
+constexpr int kGqQCol = 256;                    // first TMEM column of Q (lanes 16-31)
 
 template <int D>
 struct GqaCfg {
   static constexpr int kChunks = D / 64;           // 64-column chunks of one K or V tile
   static constexpr int kTileChunks = 2 * kChunks;  // K chunks, then V chunks
-  static constexpr int kRingTiles = D == 128 ? 6 : 12;
+  static constexpr int kRingTiles = D == 128 ? 3 : 6;
   static constexpr int kSlots = kRingTiles * kTileChunks;
-  static constexpr int kSmemBytes = kDcCtrlBytes + kSlots * kDcChunkBytes + kDcRows * 128 + 1024;
+  static constexpr int kSmemBytes = kDcCtrlBytes + kSlots * kGqChunkBytes + kGqPBytes + 1024;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -60,7 +63,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
   GqaCtrl *ctrl = reinterpret_cast<GqaCtrl *>(smem_raw);
   const uint32_t tiles_u32 = (smem_u32(smem_raw) + kDcCtrlBytes + 1023u) & ~1023u;
   const uint32_t ring_u32 = tiles_u32;                               // kRingTiles x (K, V) chunks
-  const uint32_t p_u32 = ring_u32 + Cfg::kSlots * kDcChunkBytes;     // P: 64 rows x 128 B
+  const uint32_t p_u32 = ring_u32 + Cfg::kSlots * kGqChunkBytes;     // P: two 64-key blocks
   uint8_t *p_gen = smem_raw + (p_u32 - smem_u32(smem_raw));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -92,7 +95,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     tma_prefetch_desc(&tm_v);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&ctrl->tmem_base), 256);
+    tmem_alloc(smem_u32(&ctrl->tmem_base), 512);
     tmem_relinquish();
     tc_fence_before();
   }
@@ -121,13 +124,13 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(b_tf(x), Cfg::kTileChunks * kDcChunkBytes);
+          mbar_arrive_expect_tx(b_tf(x), Cfg::kTileChunks * kGqChunkBytes);
 #pragma unroll
           for (int c = 0; c < Cfg::kChunks; ++c) {
-            tma_load_3d(ring_u32 + (x * Cfg::kTileChunks + c) * kDcChunkBytes, &tm_k, b_tf(x), c * 64, g,
-                        k0 + j * kDcKeys);
-            tma_load_3d(ring_u32 + (x * Cfg::kTileChunks + Cfg::kChunks + c) * kDcChunkBytes, &tm_v, b_tf(x), c * 64, g,
-                        k0 + j * kDcKeys);
+            tma_load_3d(ring_u32 + (x * Cfg::kTileChunks + c) * kGqChunkBytes, &tm_k, b_tf(x), c * 64, g,
+                        k0 + j * kGqKeys);
+            tma_load_3d(ring_u32 + (x * Cfg::kTileChunks + Cfg::kChunks + c) * kGqChunkBytes, &tm_v, b_tf(x), c * 64, g,
+                        k0 + j * kGqKeys);
           }
         }
       }
@@ -148,7 +151,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     auto wait_warp = [&](uint32_t bar, uint32_t parity, uint32_t site) {
       return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, hdr, site));
     };
-    constexpr uint32_t idesc_s = make_idesc_f16(BF16, kDcRows, kDcKeys, false, false);
+    constexpr uint32_t idesc_s = make_idesc_f16(BF16, kDcRows, kGqKeys, false, false);
     constexpr uint32_t idesc_o = make_idesc_f16(BF16, kDcRows, D, false, true);
     const uint32_t tmem_w = __shfl_sync(0xffffffffu, tmem, 0);
     const uint32_t s_tmem = tmem_w + (16u << 16);  // S accumulators and Q: lanes 16-31 of each sub-partition
@@ -156,8 +159,8 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     bool ok = true;
     const uint32_t k_hi = desc_hi(make_sdesc_sw128(ring_u32, 16, 1024));
     const uint32_t k_lo0 = desc_lo(make_sdesc_sw128(ring_u32, 16, 1024));
-    const uint32_t v_hi = desc_hi(make_sdesc_sw128(ring_u32, kDcChunkBytes, 1024));
-    const uint32_t v_lo0 = desc_lo(make_sdesc_sw128(ring_u32, kDcChunkBytes, 1024));
+    const uint32_t v_hi = desc_hi(make_sdesc_sw128(ring_u32, kGqChunkBytes, 1024));
+    const uint32_t v_lo0 = desc_lo(make_sdesc_sw128(ring_u32, kGqChunkBytes, 1024));
     const uint32_t p_hi = desc_hi(make_sdesc_sw128(p_u32, 16, 1024));
     const uint32_t p_lo0 = desc_lo(make_sdesc_sw128(p_u32, 16, 1024));
     // S of tile counter `t`: K-step kk into accumulator kk % 2.
@@ -165,12 +168,12 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
       const int x = t % Cfg::kRingTiles;
       if (!wait_warp(b_tf(x), (t / Cfg::kRingTiles) & 1, kDSiteSlotFull)) return false;
       tc_fence_after();
-      const uint32_t k_lo = k_lo0 + (uint32_t)((x * Cfg::kTileChunks * kDcChunkBytes) >> 4);
+      const uint32_t k_lo = k_lo0 + (uint32_t)((x * Cfg::kTileChunks * kGqChunkBytes) >> 4);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
         if (leader)
-          mma_ts2(s_tmem + (kk & 1) * kDcKeys, s_tmem + kGqQCol + kk * 8,
-                  k_lo + (uint32_t)(((kk >> 2) * kDcChunkBytes + (kk & 3) * 32) >> 4), k_hi, idesc_s,
+          mma_ts2(s_tmem + (kk & 1) * kGqKeys, s_tmem + kGqQCol + kk * 8,
+                  k_lo + (uint32_t)(((kk >> 2) * kGqChunkBytes + (kk & 3) * 32) >> 4), k_hi, idesc_s,
                   kk >= 2 ? 1u : 0u);
       if (leader) mma_commit(b_sf);
       return true;
@@ -200,12 +203,12 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
         }
         tc_fence_after();
         const uint32_t v_lo =
-            v_lo0 + (uint32_t)((((tc % Cfg::kRingTiles) * Cfg::kTileChunks + Cfg::kChunks) * kDcChunkBytes) >> 4);
+            v_lo0 + (uint32_t)((((tc % Cfg::kRingTiles) * Cfg::kTileChunks + Cfg::kChunks) * kGqChunkBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kDcKeys / 16; ++kk)
+        for (int kk = 0; kk < kGqKeys / 16; ++kk)
           if (leader)
-            mma_ss2(tmem_w, p_lo0 + (uint32_t)(kk * 2), p_hi, v_lo + (uint32_t)((kk * 16 * 128) >> 4), v_hi, idesc_o,
-                    (jj > 0 || kk > 0) ? 1u : 0u);
+            mma_ss2(tmem_w, p_lo0 + (uint32_t)(((kk >> 2) * (kDcRows * 128) + (kk & 3) * 32) >> 4), p_hi,
+                    v_lo + (uint32_t)((kk * 16 * 128) >> 4), v_hi, idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
         if (leader) {
           mma_commit(b_od);
           mma_commit(b_te(tc % Cfg::kRingTiles));
@@ -266,20 +269,29 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
           break;
         }
         tc_fence_after();
-        uint32_t sv[32], sb[32];
-        tmem_ld_half32(s_row + 0 * kDcKeys, sv);
-        tmem_ld_half32(s_row + 1 * kDcKeys, sb);
+        // This thread's 64 keys: block i in {0, 1} holds keys 64i + 32*half + e.
+        uint32_t sv[2][32];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          uint32_t sb[32];
+          tmem_ld_half32(s_row + i * 64, sv[i]);
+          tmem_ld_half32(s_row + kGqKeys + i * 64, sb);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sv[i][e] = __float_as_uint(__uint_as_float(sv[i][e]) + __uint_as_float(sb[e]));
+        }
         tc_fence_before();
         mbar_arrive(b_sx);  // S may be overwritten now
+        int lim[2];  // keys [0, lim[i]) of block i of this thread are visible
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sv[e] = __float_as_uint(__uint_as_float(sv[e]) + __uint_as_float(sb[e]));
-        const int lim = nv - j * kDcKeys - half * 32;  // keys [0, lim) of this half are visible
+        for (int i = 0; i < 2; ++i) lim[i] = nv - j * kGqKeys - i * 64 - half * 32;
         float ext = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float x = neg ? -__uint_as_float(sv[e]) : __uint_as_float(sv[e]);
-          ext = (e < lim) ? fmaxf(ext, x) : ext;
-        }
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float x = neg ? -__uint_as_float(sv[i][e]) : __uint_as_float(sv[i][e]);
+            ext = (e < lim[i]) ? fmaxf(ext, x) : ext;
+          }
         ext = fmaxf(ext, __shfl_xor_sync(0xffffffffu, ext, 16));
         const float m_tile = (ext == -INFINITY) ? -INFINITY : (neg ? -ext : ext) * c;
         const float m_new = fmaxf(m_used, m_tile);
@@ -293,17 +305,19 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
           need = true;
         }
         const float base = (m_used == -INFINITY) ? 0.f : m_used;
-        uint32_t pk[16];
+        uint32_t pk[2][16];
         float rs = 0.f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), c, -base));
-          float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, -base));
-          p0 = (2 * e < lim) ? p0 : 0.f;
-          p1 = (2 * e + 1 < lim) ? p1 : 0.f;
-          rs += p0 + p1;
-          pk[e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
-        }
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float p0 = ex2(fmaf(__uint_as_float(sv[i][2 * e]), c, -base));
+            float p1 = ex2(fmaf(__uint_as_float(sv[i][2 * e + 1]), c, -base));
+            p0 = (2 * e < lim[i]) ? p0 : 0.f;
+            p1 = (2 * e + 1 < lim[i]) ? p1 : 0.f;
+            rs += p0 + p1;
+            pk[i][e] = BF16 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+          }
         l = l * alpha + rs;
         // P (single buffer) and O may be touched only once the previous P.V is done.
         if (g > 0) {
@@ -326,12 +340,17 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
           }
           tmem_wait_st();
         }
-        // P row r, keys half*32 .. half*32+31: four 16-byte chunks, 128B swizzle.
-        uint8_t *prow = p_gen + r * 128;
+        // P row r, block i (keys 64i..64i+63, 64 rows x 128 B, 128B swizzle):
+        // this thread's keys 32*half.. are four 16-byte chunks of the row.
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int chunk = (half * 4 + i) ^ (r & 7);
-          *reinterpret_cast<uint4 *>(prow + chunk * 16) = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        for (int i = 0; i < 2; ++i) {
+          uint8_t *prow = p_gen + i * (kDcRows * 128) + r * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (half * 4 + q) ^ (r & 7);
+            *reinterpret_cast<uint4 *>(prow + chunk * 16) =
+                make_uint4(pk[i][4 * q], pk[i][4 * q + 1], pk[i][4 * q + 2], pk[i][4 * q + 3]);
+          }
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -391,7 +410,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 

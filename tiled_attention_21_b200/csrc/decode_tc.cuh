@@ -61,6 +61,7 @@ constexpr int kDcMaxGrid = 256;
 // grouped-query decode (the G = Hq/Hkv query heads of KV head g).
 struct DecodeSched {
   int heads;       // KV heads per batch entry that form separate sequences
+  int keys;        // keys per KV tile
   int *n_tiles;    // [batch*heads] KV tiles per sequence
   int *tile_pre;   // [batch*heads + 1] prefix of n_tiles
   int *seg_base;   // [batch*heads + 1] first segment of each sequence
@@ -101,7 +102,7 @@ __device__ __forceinline__ int dc_lower_bound(const int4 *segs, int n, int x) {
 
 // ----------------------------------------------------------------------------
 // Schedule: one 1024-thread CTA.
-//   n_tiles[b]   = ceil(kv_len_b / 64) (0 when the sequence has no queries)
+//   n_tiles[b]   = ceil(kv_len_b / keys) (0 when the sequence has no queries)
 //   tile_pre     = prefix of n_tiles (the global tile sequence)
 //   pieces       = num_splits > 0: min(k, n_b) near-equal pieces per sequence;
 //                  automatic: whole sequences, unless cutting the global tile
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     int n = 0;
     if (b < B) {
       const int e = b / s.heads;  // batch entry of sequence b
-      n = (p.cu_k[e + 1] - p.cu_k[e] + kDcKeys - 1) / kDcKeys;
+      n = (p.cu_k[e + 1] - p.cu_k[e] + s.keys - 1) / s.keys;
       if (p.cu_q[e + 1] - p.cu_q[e] <= 0) n = 0;  // no queries: nothing to compute
       s.n_tiles[b] = n;
       atomicMax(&max_n, n);

@@ -310,9 +310,9 @@ struct DecodeWs {
   size_t n_tiles, tile_pre, seg_base, seg_cnt, segs, part_ml, part_acc, total;
   int max_segs;
 };
-DecodeWs decode_ws(int batch, int max_kv_len, int num_splits, int dv) {
+DecodeWs decode_ws(int batch, int max_kv_len, int num_splits, int dv, int keys) {
   DecodeWs w;
-  const int tiles = (max_kv_len + kDcKeys - 1) / kDcKeys;
+  const int tiles = (max_kv_len + keys - 1) / keys;
   w.max_segs = num_splits > 0 ? batch * std::max(1, std::min(num_splits, tiles)) : batch + kDcMaxGrid;
   w.n_tiles = sizeof(WsHeader);
   w.tile_pre = w.n_tiles + align256(sizeof(int) * (size_t)batch);
@@ -340,11 +340,12 @@ bool decode_gqa_eligible(mxfa_dtype_t dt, int Hq, int Hkv, int Dqk, int Dv, int 
 }
 
 // Split schedule in the workspace for `heads` decode sequences per batch entry.
-DecodeSched decode_sched(const AttnParams &p, int heads, int num_splits, int dv, void *ws, int sms) {
-  const DecodeWs w = decode_ws(p.batch * heads, p.max_sk, num_splits, dv);
+DecodeSched decode_sched(const AttnParams &p, int heads, int num_splits, int dv, int keys, void *ws, int sms) {
+  const DecodeWs w = decode_ws(p.batch * heads, p.max_sk, num_splits, dv, keys);
   char *base = static_cast<char *>(ws);
   DecodeSched s;
   s.heads = heads;
+  s.keys = keys;
   s.n_tiles = reinterpret_cast<int *>(base + w.n_tiles);
   s.tile_pre = reinterpret_cast<int *>(base + w.tile_pre);
   s.seg_base = reinterpret_cast<int *>(base + w.seg_base);
@@ -363,10 +364,10 @@ mxfa_status_t launch_decode_gqa_t(AttnParams &p, mxfa_dtype_t dt, int total_kv, 
                                   cudaStream_t st) {
   int sms = 0;
   MXFA_TRY(sm_count(&sms));
-  const DecodeSched s = decode_sched(p, p.hkv, num_splits, D, ws, sms);
+  const DecodeSched s = decode_sched(p, p.hkv, num_splits, D, kGqKeys, ws, sms);
   CUtensorMap mk, mv;
-  MXFA_TRY(make_map(&mk, p.k, dt, D, p.hkv, total_kv, p.k_rs, p.k_hs, kDcKeys));
-  MXFA_TRY(make_map(&mv, p.v, dt, D, p.hkv, total_kv, p.v_rs, p.v_hs, kDcKeys));
+  MXFA_TRY(make_map(&mk, p.k, dt, D, p.hkv, total_kv, p.k_rs, p.k_hs, kGqKeys));
+  MXFA_TRY(make_map(&mv, p.v, dt, D, p.hkv, total_kv, p.v_rs, p.v_hs, kGqKeys));
   decode_prep_kernel<<<1, 1024, 0, st>>>(p, s);
   MXFA_CUDA(cudaGetLastError());
   auto k = attn_decode_gqa_kernel<D, BF16>;
@@ -393,7 +394,7 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
                                cudaStream_t st) {
   int sms = 0;
   MXFA_TRY(sm_count(&sms));
-  const DecodeSched s = decode_sched(p, 1, num_splits, kDcDv, ws, sms);
+  const DecodeSched s = decode_sched(p, 1, num_splits, kDcDv, kDcKeys, ws, sms);
   CUtensorMap mq, mkv;
   MXFA_TRY(make_map_2d(&mq, p.q, dt, kDcDqk, (int64_t)total_q * p.hq, kDcDqk));
   MXFA_TRY(make_map_2d(&mkv, p.k, dt, kDcDqk, total_kv, p.k_rs));
@@ -545,9 +546,9 @@ size_t mxfa_attn_decode_splitkv_workspace_size(int batch, int max_q_len, int Hq,
                                                int num_splits, mxfa_dtype_t dtype) {
   if (dtype == MXFA_F32 || batch <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || num_splits < 0) return sizeof(WsHeader);
   if (Dv == kDcDv && Hkv == 1 && (int64_t)max_q_len * Hq <= kDcRows)  // MLA
-    return decode_ws(batch, max_kv_len, num_splits, kDcDv).total;
+    return decode_ws(batch, max_kv_len, num_splits, kDcDv, kDcKeys).total;
   if ((Dv == 64 || Dv == 128) && (int64_t)max_q_len * (Hq / Hkv) <= kDcRows)  // grouped-query heads
-    return decode_ws(batch * Hkv, max_kv_len, num_splits, Dv).total;
+    return decode_ws(batch * Hkv, max_kv_len, num_splits, Dv, kGqKeys).total;
   return sizeof(WsHeader);
 }
 
