@@ -55,9 +55,11 @@ def prefill_flops(B, H, S, D, causal=True):
 
 
 def decode_bytes(p):
-    """Algorithmic bytes of one MLA decode: the KV cache once, q, O and LSE."""
+    """Algorithmic bytes of one decode: the KV cache once (MLA: the shared
+    latent rows; grouped-query: K and V), q, O and LSE."""
     es = 2
-    return (p.kv.numel() * es + p.q.numel() * es + p.total_q * p.hq * p.dv * es + p.total_q * p.hq * 4)
+    kv = p.kv.numel() * es if p.mla else (p.k.numel() + p.v.numel()) * es
+    return kv + p.q.numel() * es + p.total_q * p.hq * p.dv * es + p.total_q * p.hq * 4
 
 
 def kernel_hash():
@@ -239,7 +241,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=128,
                     help="sequences of the MLA decode workload (128 = the full workload; smaller for captures)")
-    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "gqa"], default=None,
                     help="time one workload only (used for profiling captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -278,7 +280,7 @@ def main():
         mx.mxfa_attn_fwd(q, k, v, causal=True, out=o, lse=lse, ws=ws, stream=stream)
 
     flops = prefill_flops(B, H, S, D)
-    if args.only == "decode":
+    if args.only in ("decode", "gqa"):
         args.steps = 0
     with ClockSampler(local) as clk:
         times = time_steps(step, args.steps, args.warmup, flush, stream, world)
@@ -319,7 +321,7 @@ def main():
 
     # ---------------- decode (secondary measurement)
     decode = None
-    if not args.no_decode and args.only != "prefill":
+    if not args.no_decode and args.only in (None, "decode"):
         pdc = (workloads.cfg_mla_decode() if args.decode_batch == 128 else
                workloads.mla_decode(3, args.decode_batch, 4, 8192, name=f"mla_decode_b{args.decode_batch}_q4_h16_kv8192_bf16"))
         dd = to_dev(pdc, dev)
@@ -344,6 +346,32 @@ def main():
                                "traffic": recorded_traffic("decode", "mla_decode_b128_q4_h16_kv8192_bf16"),
                                "peak_kind": f"{pk_kind} HBM copy"}}
 
+    # ---------------- grouped-query decode (next scope row; secondary measurement)
+    decode_gqa = None
+    if not args.no_decode and args.only in (None, "gqa"):
+        pg = workloads.cfg_gqa_decode()
+        dg = to_dev(pg, dev)
+        og = torch.empty((pg.total_q, pg.hq, pg.dv), dtype=torch.bfloat16, device=dev)
+        lg = torch.empty((pg.total_q, pg.hq), dtype=torch.float32, device=dev)
+        kvl = pg.total_k // pg.batch
+        need = mx.load().mxfa_attn_decode_splitkv_workspace_size(pg.batch, 1, pg.hq, pg.hkv, pg.dv, kvl, 0, 2)
+        wsg = torch.zeros(need + 256, dtype=torch.uint8, device=dev)
+
+        def gstep():
+            mx.mxfa_attn_decode_splitkv(dg["q"], dg["k"], dg["v"], dg["cu_q"], dg["cu_k"], 1, kvl,
+                                        softmax_scale=pg.scale, out=og, lse=lg, ws=wsg, stream=stream)
+
+        gtimes = time_steps(gstep, max(5, args.steps // 3), 3, lambda: None, stream, world)  # KV 1.07 GB >> L2
+        gbytes = decode_bytes(pg)
+        gms = max_over_ranks(statistics.mean(gtimes), world)
+        ggbs = gbytes / (gms / 1e3) / 1e9
+        decode_gqa = {"workload": pg.name, "value": ggbs * world, "unit": "GB/s", "ms_per_step": gms,
+                      "algorithmic_bytes": gbytes, "l2": "inputs (1.07 GB K+V) larger than L2",
+                      "roofline": {"bound": "hbm", "achieved": ggbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                   "frac": ggbs / pk["hbm_gbs"],
+                                   "traffic": recorded_traffic("decode_gqa", pg.name),
+                                   "peak_kind": f"{pk_kind} HBM copy"}}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only is None:
         cpu = cpu_baseline_prefill()
@@ -358,7 +386,8 @@ def main():
                 "roofline": roofline, "cpu_baseline": cpu,
                 "e2e": None if args.only else {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                                                "d2h_bytes_per_step": d2h},
-                "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode}
+                "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
+                "decode_gqa": decode_gqa}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
