@@ -174,6 +174,41 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
                                        mxfa_dtype_t dtype, float softmax_scale, int causal, int num_splits,
                                        void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Decode over a KV cache, with an optional append (mxflashattn 1.4.0 api.py,
+ * flash_attn_with_kvcache: q, k_cache, v_cache, k, v, cache_seqlens,
+ * block_table, causal).
+ *   q: [batch, Sq, Hq, D] contiguous, bf16 or f16, D = 64 or 128,
+ *      Sq * (Hq / Hkv) <= 64 (otherwise MXFA_ERR_UNSUPPORTED).
+ *   k_cache, v_cache: [num_pages, page_size, Hkv, D] contiguous.  Dense cache
+ *      (block_table == NULL): num_pages = batch, page_size = the cache length,
+ *      key position pos of batch entry b is row b*page_size + pos.  Paged
+ *      cache: block_table [batch, max_blocks_per_seq] int32 (device) gives the
+ *      page of key positions [i*page_size, (i+1)*page_size) of entry b;
+ *      page_size is a power of two in [16, 128] or a multiple of 128.
+ *   cache_seqlens: [batch] int32 (device), keys already cached per entry.
+ *   k_new, v_new: [batch, Snew, Hkv, D] contiguous or both NULL (Snew = 0).
+ *      Row i of entry b is written to key position cache_seqlens[b] + i
+ *      before the attention, and cache_seqlens[b] is then advanced by Snew
+ *      in place (a position beyond the cache's capacity is not written and
+ *      the workspace status reports MXFA_ERR_INVALID_ARG).
+ *   Attention: query i of entry b (of Sq) sees key positions [0, L_b),
+ *      L_b = cache_seqlens[b] + Snew (as passed in); causal: j <= i + L_b - Sq.
+ *   o: [batch, Sq, Hq, D] contiguous; lse: [batch, Sq, Hq] fp32 (or NULL).
+ *   max_len: an upper bound of every L_b (sizes the workspace schedule).
+ *   num_splits: as for mxfa_attn_decode_splitkv.
+ * The caller owns every buffer; the library writes k_cache / v_cache only at
+ * the appended positions and cache_seqlens only by the advance.
+ */
+size_t mxfa_attn_decode_kvcache_workspace_size(int batch, int Sq, int Hq, int Hkv, int D, int max_len,
+                                               int num_splits, mxfa_dtype_t dtype);
+mxfa_status_t mxfa_attn_decode_kvcache(const void *q, void *k_cache, void *v_cache, const void *k_new,
+                                       const void *v_new, int32_t *cache_seqlens, const int32_t *block_table,
+                                       int batch, int Sq, int Snew, int Hq, int Hkv, int D, int num_pages,
+                                       int page_size, int max_blocks_per_seq, int max_len, mxfa_dtype_t dtype,
+                                       float softmax_scale, int causal, int num_splits, void *o, float *lse,
+                                       void *workspace, size_t workspace_bytes, void *stream);
+
 /* Message for the calling thread's most recent failure ("" if none). */
 const char *mxfa_last_error(void);
 

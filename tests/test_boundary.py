@@ -118,3 +118,31 @@ def test_product_path_does_not_touch_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower(), f
+
+
+def test_kvcache_validation(lib):
+    import tiled_attention_21_b200 as m
+    call = lib.mxfa_attn_decode_kvcache
+
+    def c(**kw):
+        a = dict(q=FAKE, kc=FAKE, vc=FAKE, kn=None, vn=None, sl=FAKE, bt=FAKE, B=2, Sq=1, Snew=0, Hq=32, Hkv=4, D=128,
+                 pages=8, page=64, blocks=4, max_len=256, dt=2, scale=float("nan"), causal=0, splits=0, o=FAKE,
+                 lse=None, ws=FAKE, wn=1 << 20)
+        a.update(kw)
+        return call(a["q"], a["kc"], a["vc"], a["kn"], a["vn"], a["sl"], a["bt"], a["B"], a["Sq"], a["Snew"],
+                    a["Hq"], a["Hkv"], a["D"], a["pages"], a["page"], a["blocks"], a["max_len"], a["dt"], a["scale"],
+                    a["causal"], a["splits"], a["o"], a["lse"], a["ws"], a["wn"], None)
+
+    assert c(D=96) == m.MXFA_ERR_UNSUPPORTED                 # head dim
+    assert c(dt=0) == m.MXFA_ERR_UNSUPPORTED                 # fp32
+    assert c(Sq=16) == m.MXFA_ERR_UNSUPPORTED                # 16 * 8 query rows per KV head > 64
+    assert c(page=48) == m.MXFA_ERR_UNSUPPORTED              # page size
+    assert c(Hq=30) == m.MXFA_ERR_INVALID_ARG                # Hq not a multiple of Hkv
+    assert c(Snew=2) == m.MXFA_ERR_INVALID_ARG               # appended rows without k_new / v_new
+    assert c(sl=None) == m.MXFA_ERR_INVALID_ARG              # cache_seqlens missing
+    assert c(bt=None, pages=3) == m.MXFA_ERR_INVALID_ARG     # dense cache: one page per batch entry
+    assert c(blocks=0) == m.MXFA_ERR_INVALID_ARG             # empty block table
+    assert c(wn=16) == m.MXFA_ERR_WORKSPACE                  # workspace too small
+    assert c(B=0) == m.MXFA_OK                               # nothing to do
+    need = lib.mxfa_attn_decode_kvcache_workspace_size(64, 1, 32, 4, 128, 8192, 0, 2)
+    assert need > 256 and need == lib.mxfa_attn_decode_splitkv_workspace_size(64, 1, 32, 4, 128, 8192, 0, 2)

@@ -56,6 +56,10 @@ def load():
             lib.mxfa_attn_decode_splitkv.restype = i32
             lib.mxfa_attn_decode_splitkv_workspace_size.argtypes = [i32] * 8
             lib.mxfa_attn_decode_splitkv_workspace_size.restype = sz
+            lib.mxfa_attn_decode_kvcache.argtypes = [vp] * 7 + [i32] * 10 + [i32, f32, i32, i32, vp, vp, vp, sz, vp]
+            lib.mxfa_attn_decode_kvcache.restype = i32
+            lib.mxfa_attn_decode_kvcache_workspace_size.argtypes = [i32] * 8
+            lib.mxfa_attn_decode_kvcache_workspace_size.restype = sz
             lib.mxfa_last_error.argtypes = []
             lib.mxfa_last_error.restype = ctypes.c_char_p
             lib.mxfa_read_device_status.argtypes = [vp, vp]
@@ -203,5 +207,44 @@ def mxfa_attn_decode_splitkv(q, k, v, qo_indptr, kv_indptr, max_q_len: int, max_
     return out, lse
 
 
-__all__ = ["load", "mxfa_attn_fwd", "mxfa_attn_varlen_fwd", "mxfa_attn_decode_splitkv", "read_device_status",
-           "workspace", "MxfaError", "LIB_PATH"]
+def mxfa_attn_decode_kvcache(q, k_cache, v_cache, cache_seqlens, k_new=None, v_new=None, block_table=None,
+                             softmax_scale: float | None = None, causal: bool = False, num_splits: int = 0,
+                             max_len: int | None = None, out=None, lse=None, return_lse: bool = True,
+                             ws: torch.Tensor | None = None, stream=None):
+    """Decode over a KV cache.  q [B, Sq, Hq, D]; k_cache / v_cache [B, cache_len,
+    Hkv, D] (dense, block_table None) or [num_pages, page_size, Hkv, D] with
+    block_table [B, max_blocks] int32 (paged); cache_seqlens [B] int32 on the
+    device.  k_new / v_new [B, Snew, Hkv, D] are appended at cache_seqlens
+    first, and cache_seqlens is advanced by Snew in place.  All contiguous.
+    Returns (o [B, Sq, Hq, D], lse [B, Sq, Hq])."""
+    lib = load()
+    B, Sq, Hq, D = q.shape
+    num_pages, page_size, Hkv, _ = k_cache.shape
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("k_new", k_new), ("v_new", v_new),
+                    ("cache_seqlens", cache_seqlens), ("block_table", block_table)):
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if cache_seqlens.dtype != torch.int32 or (block_table is not None and block_table.dtype != torch.int32):
+        raise ValueError("cache_seqlens and block_table must be int32")
+    Snew = 0 if k_new is None else k_new.shape[1]
+    max_blocks = 0 if block_table is None else block_table.shape[1]
+    if max_len is None:
+        max_len = page_size * max_blocks if block_table is not None else page_size
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Sq, Hq), dtype=torch.float32, device=q.device)
+    dt = _DT[q.dtype]
+    need = lib.mxfa_attn_decode_kvcache_workspace_size(B, Sq, Hq, Hkv, D, int(max_len), num_splits, dt)
+    ws = ws if ws is not None else workspace(need, q.device)
+    wp, wn = _ws_view(ws)
+    _check(lib.mxfa_attn_decode_kvcache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_new), _ptr(v_new),
+                                        _ptr(cache_seqlens), _ptr(block_table), B, Sq, Snew, Hq, Hkv, D, num_pages,
+                                        page_size, max_blocks, int(max_len), dt, _scale(softmax_scale),
+                                        int(bool(causal)), int(num_splits), _ptr(out), _ptr(lse), wp, wn,
+                                        _stream(stream)))
+    return out, lse
+
+
+__all__ = ["load", "mxfa_attn_fwd", "mxfa_attn_varlen_fwd", "mxfa_attn_decode_splitkv", "mxfa_attn_decode_kvcache",
+           "read_device_status", "workspace", "MxfaError", "LIB_PATH"]

@@ -117,7 +117,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
       for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
         const int4 sd = s.segs[sg];
         const int b = sd.x / s.heads, g = sd.x % s.heads;
-        const int k0 = p.cu_k[b];
+        const int len = dc_klen(p, s, b);
         for (int j = sd.y; ok && j < sd.z; ++j, ++tc) {
           const int x = tc % Cfg::kRingTiles;
           if (!wait_bar(b_te(x), ((tc / Cfg::kRingTiles) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty)) {
@@ -125,12 +125,20 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
             break;
           }
           mbar_arrive_expect_tx(b_tf(x), Cfg::kTileChunks * kGqChunkBytes);
+          // A tile is one box of 128 rows when its keys are contiguous rows
+          // (packed or dense), else one box per cache page of it (the maps'
+          // box height is then the page size, a divisor of 128).
+          const int box = (p.cu_k || !s.block_table || s.page_size >= kGqKeys) ? kGqKeys : s.page_size;
+          for (int i = 0; i < kGqKeys / box; ++i) {
+            const int pos = j * kGqKeys + i * box;
+            const int row = pos < len ? dc_krow(p, s, b, pos) : -(1 << 30);
 #pragma unroll
-          for (int c = 0; c < Cfg::kChunks; ++c) {
-            tma_load_3d(ring_u32 + (x * Cfg::kTileChunks + c) * kGqChunkBytes, &tm_k, b_tf(x), c * 64, g,
-                        k0 + j * kGqKeys);
-            tma_load_3d(ring_u32 + (x * Cfg::kTileChunks + Cfg::kChunks + c) * kGqChunkBytes, &tm_v, b_tf(x), c * 64, g,
-                        k0 + j * kGqKeys);
+            for (int c = 0; c < Cfg::kChunks; ++c) {
+              tma_load_3d(ring_u32 + (x * Cfg::kTileChunks + c) * kGqChunkBytes + i * box * 128, &tm_k, b_tf(x), c * 64,
+                          g, row);
+              tma_load_3d(ring_u32 + (x * Cfg::kTileChunks + Cfg::kChunks + c) * kGqChunkBytes + i * box * 128, &tm_v,
+                          b_tf(x), c * 64, g, row);
+            }
           }
         }
       }
@@ -233,7 +241,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     // thread writes half `half` of row r.
     auto load_q = [&](int sg) {
       const int v = s.segs[sg].x, b = v / s.heads, gh = v % s.heads;
-      const int q0 = p.cu_q[b], rows = (p.cu_q[b + 1] - q0) * G;
+      const int q0 = dc_q(p, b).x, rows = dc_q(p, b).y * G;
       const bool vq = r < rows;
       const uint4 *src = reinterpret_cast<const uint4 *>(
           reinterpret_cast<const uint16_t *>(p.q) +
@@ -256,7 +264,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
       const int4 sd = s.segs[sg];
       const int v = sd.x, b = v / s.heads, gh = v % s.heads;
-      const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0, sk = p.cu_k[b + 1] - p.cu_k[b];
+      const int q0 = dc_q(p, b).x, sq = dc_q(p, b).y, sk = dc_klen(p, s, b);
       const int rows = sq * G;
       const bool valid = r < rows;
       const int nv = valid ? visible_keys(r / G, sq, sk, p.causal) : 0;
@@ -411,6 +419,39 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// KV-cache append (the k / v arguments of mxflashattn flash_attn_with_kvcache):
+// row i of batch entry b of k_new / v_new ([B, snew, Hkv, D]) goes to key
+// position cache_seqlens[b] + i of the cache, before the attention reads it.
+// Block (i, b); each thread copies 16-byte pieces of the Hkv*D values.  A
+// position past the cache's capacity, or a page outside the pool, is not
+// written; the call then reports MXFA_ERR_INVALID_ARG in the workspace.
+__global__ void __launch_bounds__(256) kv_append_kernel(const AttnParams p, const DecodeSched s, const void *k_new,
+                                                         const void *v_new, int snew, int num_rows) {
+  const int i = blockIdx.x, b = blockIdx.y;
+  const int pos = s.cache_seqlens[b] + i;
+  int row;
+  if (!s.block_table) {
+    row = (pos >= 0 && pos < s.page_size) ? b * s.page_size + pos : -1;
+  } else {
+    const int idx = pos / s.page_size;
+    const int page = (pos >= 0 && idx < s.max_blocks) ? s.block_table[(int64_t)b * s.max_blocks + idx] : -1;
+    row = page >= 0 ? page * s.page_size + pos % s.page_size : -1;
+  }
+  if (row < 0 || row >= num_rows) {
+    if (threadIdx.x == 0) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x501);
+    return;
+  }
+  const int per_row = p.hkv * p.dqk / 8;  // 16-byte pieces of one token's K (or V)
+  const uint4 *ks = reinterpret_cast<const uint4 *>(k_new) + ((int64_t)b * snew + i) * per_row;
+  const uint4 *vs = reinterpret_cast<const uint4 *>(v_new) + ((int64_t)b * snew + i) * per_row;
+  for (int t = threadIdx.x; t < per_row; t += blockDim.x) {
+    const int g = t / (p.dqk / 8), c = t % (p.dqk / 8);
+    reinterpret_cast<uint4 *>(const_cast<void *>(p.k))[((int64_t)row * p.k_rs + (int64_t)g * p.k_hs) / 8 + c] = ks[t];
+    reinterpret_cast<uint4 *>(const_cast<void *>(p.v))[((int64_t)row * p.v_rs + (int64_t)g * p.v_hs) / 8 + c] = vs[t];
   }
 }
 

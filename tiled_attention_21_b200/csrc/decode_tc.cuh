@@ -72,7 +72,38 @@ struct DecodeSched {
   int max_segs;
   int num_splits;  // 0 = automatic
   int grid;
+  // KV-cache mode (p.cu_k == nullptr): batch entry b has cache_seqlens[b] + add
+  // keys; key position pos is cache row b*page_size + pos (dense cache,
+  // block_table == nullptr) or block_table[b][pos / page_size]*page_size +
+  // pos % page_size (paged).  The prep kernel writes the key counts to
+  // kv_len and, when advance != 0, then adds `add` to cache_seqlens.
+  int32_t *cache_seqlens;
+  int add, advance;
+  int *kv_len;
+  const int32_t *block_table;
+  int max_blocks, page_size;
 };
+
+// Queries of batch entry b: (first row, count); packed (cu_q) or uniform.
+__device__ __forceinline__ int2 dc_q(const AttnParams &p, int b) {
+  if (p.cu_q) return make_int2(p.cu_q[b], p.cu_q[b + 1] - p.cu_q[b]);
+  return make_int2(b * p.max_sq, p.max_sq);
+}
+// Keys of batch entry b.
+__device__ __forceinline__ int dc_klen(const AttnParams &p, const DecodeSched &s, int b) {
+  return p.cu_k ? p.cu_k[b + 1] - p.cu_k[b] : s.kv_len[b];
+}
+// Cache row of key position pos (< its key count) of batch entry b, or an
+// out-of-range row (read as zeros by TMA) when the block table has no page
+// for it.
+__device__ __forceinline__ int dc_krow(const AttnParams &p, const DecodeSched &s, int b, int pos) {
+  if (p.cu_k) return p.cu_k[b] + pos;
+  if (!s.block_table) return b * s.page_size + pos;
+  const int idx = pos / s.page_size;
+  if (idx >= s.max_blocks) return -(1 << 30);
+  const int page = s.block_table[(int64_t)b * s.max_blocks + idx];
+  return page < 0 ? -(1 << 30) : page * s.page_size + pos % s.page_size;
+}
 
 struct DecodeCtrl {
   uint64_t q_ready;
@@ -125,8 +156,10 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     int n = 0;
     if (b < B) {
       const int e = b / s.heads;  // batch entry of sequence b
-      n = (p.cu_k[e + 1] - p.cu_k[e] + s.keys - 1) / s.keys;
-      if (p.cu_q[e + 1] - p.cu_q[e] <= 0) n = 0;  // no queries: nothing to compute
+      const int len = p.cu_k ? p.cu_k[e + 1] - p.cu_k[e] : s.cache_seqlens[e] + s.add;
+      if (!p.cu_k && b % s.heads == 0) s.kv_len[e] = len;
+      n = (len + s.keys - 1) / s.keys;
+      if (dc_q(p, e).y <= 0) n = 0;  // no queries: nothing to compute
       s.n_tiles[b] = n;
       atomicMax(&max_n, n);
     }
@@ -139,6 +172,8 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
   }
   if (tid == 0) s.tile_pre[0] = 0;
   const int T = carry;
+  if (!p.cu_k && s.advance)  // every read of cache_seqlens above is done
+    for (int e = tid; e < p.batch; e += 1024) s.cache_seqlens[e] += s.add;
   for (int c = tid; c <= G; c += 1024) cut[c] = (int)(((int64_t)c * T) / G);
   if (tid == 0) {
     // longest CTA with whole sequences (they are dealt out by first tile) vs. the even cut
@@ -589,7 +624,8 @@ template <typename T, int DV>
 __global__ void __launch_bounds__(DV / 4) decode_combine_kernel(const AttnParams p, const DecodeSched s) {
   const int r = blockIdx.x, v = blockIdx.y;
   const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
-  const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
+  const int2 qr = dc_q(p, b);
+  const int q0 = qr.x, sq = qr.y;
   if (r >= sq * G) return;
   const int cnt = s.seg_cnt[v];
   if (cnt == 1) return;  // stored directly by the decode kernel

@@ -307,7 +307,7 @@ mxfa_status_t prefill(AttnParams &p, mxfa_dtype_t dt, int D, bool varlen, int64_
 // sequences (batch entries x KV heads that form separate sequences), Dv
 // output columns.
 struct DecodeWs {
-  size_t n_tiles, tile_pre, seg_base, seg_cnt, segs, part_ml, part_acc, total;
+  size_t n_tiles, tile_pre, seg_base, seg_cnt, kv_len, segs, part_ml, part_acc, total;
   int max_segs;
 };
 DecodeWs decode_ws(int batch, int max_kv_len, int num_splits, int dv, int keys) {
@@ -318,7 +318,8 @@ DecodeWs decode_ws(int batch, int max_kv_len, int num_splits, int dv, int keys) 
   w.tile_pre = w.n_tiles + align256(sizeof(int) * (size_t)batch);
   w.seg_base = w.tile_pre + align256(sizeof(int) * (size_t)(batch + 1));
   w.seg_cnt = w.seg_base + align256(sizeof(int) * (size_t)(batch + 1));
-  w.segs = w.seg_cnt + align256(sizeof(int) * (size_t)batch);
+  w.kv_len = w.seg_cnt + align256(sizeof(int) * (size_t)batch);
+  w.segs = w.kv_len + align256(sizeof(int) * (size_t)batch);
   w.part_ml = w.segs + align256(sizeof(int4) * (size_t)w.max_segs);
   w.part_acc = w.part_ml + align256(sizeof(float2) * (size_t)w.max_segs * kDcRows);
   w.total = w.part_acc + align256(sizeof(float) * (size_t)w.max_segs * kDcRows * dv);
@@ -353,21 +354,25 @@ DecodeSched decode_sched(const AttnParams &p, int heads, int num_splits, int dv,
   s.segs = reinterpret_cast<int4 *>(base + w.segs);
   s.part_ml = reinterpret_cast<float2 *>(base + w.part_ml);
   s.part_acc = reinterpret_cast<float *>(base + w.part_acc);
+  s.kv_len = reinterpret_cast<int *>(base + w.kv_len);
   s.max_segs = w.max_segs;
   s.num_splits = num_splits;
   s.grid = std::min(sms, kDcMaxGrid);
+  s.cache_seqlens = nullptr;
+  s.add = s.advance = 0;
+  s.block_table = nullptr;
+  s.max_blocks = s.page_size = 0;
   return s;
 }
 
+// `kv_rows`: rows of the K / V tensors; `box`: TMA box height (128, or the
+// page size of a paged cache with pages shorter than a tile).
 template <int D, bool BF16>
-mxfa_status_t launch_decode_gqa_t(AttnParams &p, mxfa_dtype_t dt, int total_kv, int num_splits, void *ws,
+mxfa_status_t launch_decode_gqa_t(AttnParams &p, const DecodeSched &s, mxfa_dtype_t dt, int64_t kv_rows, int box,
                                   cudaStream_t st) {
-  int sms = 0;
-  MXFA_TRY(sm_count(&sms));
-  const DecodeSched s = decode_sched(p, p.hkv, num_splits, D, kGqKeys, ws, sms);
   CUtensorMap mk, mv;
-  MXFA_TRY(make_map(&mk, p.k, dt, D, p.hkv, total_kv, p.k_rs, p.k_hs, kGqKeys));
-  MXFA_TRY(make_map(&mv, p.v, dt, D, p.hkv, total_kv, p.v_rs, p.v_hs, kGqKeys));
+  MXFA_TRY(make_map(&mk, p.k, dt, D, p.hkv, kv_rows, p.k_rs, p.k_hs, box));
+  MXFA_TRY(make_map(&mv, p.v, dt, D, p.hkv, kv_rows, p.v_rs, p.v_hs, box));
   decode_prep_kernel<<<1, 1024, 0, st>>>(p, s);
   MXFA_CUDA(cudaGetLastError());
   auto k = attn_decode_gqa_kernel<D, BF16>;
@@ -380,14 +385,14 @@ mxfa_status_t launch_decode_gqa_t(AttnParams &p, mxfa_dtype_t dt, int total_kv, 
   return MXFA_OK;
 }
 
-mxfa_status_t launch_decode_gqa(AttnParams &p, mxfa_dtype_t dt, int total_kv, int num_splits, void *ws,
+mxfa_status_t launch_decode_gqa(AttnParams &p, const DecodeSched &s, mxfa_dtype_t dt, int64_t kv_rows, int box,
                                 cudaStream_t st) {
   const bool bf = dt == MXFA_BF16;
   if (p.dqk == 128)
-    return bf ? launch_decode_gqa_t<128, true>(p, dt, total_kv, num_splits, ws, st)
-              : launch_decode_gqa_t<128, false>(p, dt, total_kv, num_splits, ws, st);
-  return bf ? launch_decode_gqa_t<64, true>(p, dt, total_kv, num_splits, ws, st)
-            : launch_decode_gqa_t<64, false>(p, dt, total_kv, num_splits, ws, st);
+    return bf ? launch_decode_gqa_t<128, true>(p, s, dt, kv_rows, box, st)
+              : launch_decode_gqa_t<128, false>(p, s, dt, kv_rows, box, st);
+  return bf ? launch_decode_gqa_t<64, true>(p, s, dt, kv_rows, box, st)
+            : launch_decode_gqa_t<64, false>(p, s, dt, kv_rows, box, st);
 }
 
 mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int total_kv, int num_splits, void *ws,
@@ -602,9 +607,94 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
   p.pairs = nullptr;
   if (decode_tc_eligible(dtype, Hq, Hkv, Dqk, Dv, max_q_len, k, v, k_row_stride, v_row_stride) && total_kv > 0)
     return launch_decode_tc(p, dtype, total_q, total_kv, num_splits, workspace, st);
-  if (decode_gqa_eligible(dtype, Hq, Hkv, Dqk, Dv, max_q_len, k_row_stride, v_row_stride) && total_kv > 0)
-    return launch_decode_gqa(p, dtype, total_kv, num_splits, workspace, st);
+  if (decode_gqa_eligible(dtype, Hq, Hkv, Dqk, Dv, max_q_len, k_row_stride, v_row_stride) && total_kv > 0) {
+    int sms = 0;
+    MXFA_TRY(sm_count(&sms));
+    const DecodeSched s = decode_sched(p, Hkv, num_splits, Dv, kGqKeys, workspace, sms);
+    return launch_decode_gqa(p, s, dtype, total_kv, kGqKeys, st);
+  }
   return launch_simt_any(dtype, p, max_q_len, st);
+}
+
+size_t mxfa_attn_decode_kvcache_workspace_size(int batch, int Sq, int Hq, int Hkv, int D, int max_len,
+                                               int num_splits, mxfa_dtype_t dtype) {
+  if (dtype == MXFA_F32 || batch <= 0 || Sq <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || num_splits < 0 ||
+      (D != 64 && D != 128) || (int64_t)Sq * (Hq / Hkv) > kDcRows || max_len < 0)
+    return sizeof(WsHeader);
+  return decode_ws(batch * Hkv, max_len, num_splits, D, kGqKeys).total;
+}
+
+mxfa_status_t mxfa_attn_decode_kvcache(const void *q, void *k_cache, void *v_cache, const void *k_new,
+                                       const void *v_new, int32_t *cache_seqlens, const int32_t *block_table,
+                                       int batch, int Sq, int Snew, int Hq, int Hkv, int D, int num_pages,
+                                       int page_size, int max_blocks_per_seq, int max_len, mxfa_dtype_t dtype,
+                                       float softmax_scale, int causal, int num_splits, void *o, float *lse,
+                                       void *workspace, size_t workspace_bytes, void *stream) {
+  if (!dtype_ok(dtype)) return fail(MXFA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (batch < 0 || Sq < 0 || Snew < 0 || num_pages < 0 || page_size <= 0 || max_len < 0 || num_splits < 0 ||
+      max_blocks_per_seq < 0)
+    return fail(MXFA_ERR_INVALID_ARG, "negative size or non-positive page size");
+  MXFA_TRY(check_heads(Hq, Hkv));
+  if (D != 64 && D != 128) return fail(MXFA_ERR_UNSUPPORTED, "head dimension %d is not 64 or 128", D);
+  if (std::isinf(softmax_scale)) return fail(MXFA_ERR_INVALID_ARG, "softmax_scale is infinite");
+  if (dtype == MXFA_F32) return fail(MXFA_ERR_UNSUPPORTED, "the KV-cache decode takes bf16 or f16");
+  if ((int64_t)Sq * (Hq / Hkv) > kDcRows)
+    return fail(MXFA_ERR_UNSUPPORTED, "Sq * Hq / Hkv = %lld query rows per KV head exceed %d",
+                (long long)Sq * (Hq / Hkv), kDcRows);
+  if ((k_new == nullptr) != (v_new == nullptr) || (Snew > 0 && k_new == nullptr))
+    return fail(MXFA_ERR_INVALID_ARG, "k_new and v_new go together, and Snew > 0 needs them");
+  if (batch == 0 || Sq == 0) return MXFA_OK;
+  if (!cache_seqlens) return fail(MXFA_ERR_INVALID_ARG, "cache_seqlens is NULL");
+  const bool paged = block_table != nullptr;
+  if (paged) {
+    const bool pow2 = (page_size & (page_size - 1)) == 0;
+    if (!((page_size >= 16 && page_size <= kGqKeys && pow2) || page_size % kGqKeys == 0))
+      return fail(MXFA_ERR_UNSUPPORTED, "page size %d: a power of two in [16, 128] or a multiple of 128", page_size);
+    if (max_blocks_per_seq <= 0) return fail(MXFA_ERR_INVALID_ARG, "block table with no columns");
+  } else if (num_pages != batch) {
+    return fail(MXFA_ERR_INVALID_ARG, "a dense cache holds one page of page_size rows per batch entry");
+  }
+  if ((int64_t)num_pages * page_size >= (1ll << 30))
+    return fail(MXFA_ERR_UNSUPPORTED, "cache of %lld rows exceeds 2^30", (long long)num_pages * page_size);
+  MXFA_TRY(check_ptr(q, "q"));
+  MXFA_TRY(check_ptr(o, "o"));
+  MXFA_TRY(check_ptr(k_cache, "k_cache"));
+  MXFA_TRY(check_ptr(v_cache, "v_cache"));
+  MXFA_TRY(check_ptr(lse, "lse", true));
+  if (k_new) {
+    MXFA_TRY(check_ptr(k_new, "k_new"));
+    MXFA_TRY(check_ptr(v_new, "v_new"));
+  }
+  MXFA_TRY(check_workspace(workspace, workspace_bytes,
+                           mxfa_attn_decode_kvcache_workspace_size(batch, Sq, Hq, Hkv, D, max_len, num_splits, dtype)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnParams p{};
+  p.q = q; p.k = k_cache; p.v = v_cache; p.o = o; p.lse = lse;
+  p.cu_q = nullptr; p.cu_k = nullptr;
+  p.batch = batch; p.max_sq = Sq; p.max_sk = max_len;
+  p.hq = Hq; p.hkv = Hkv; p.dqk = D; p.dv = D;
+  p.q_rs = (int64_t)Hq * D; p.q_hs = D;
+  p.k_rs = p.v_rs = (int64_t)Hkv * D; p.k_hs = p.v_hs = D;
+  p.o_rs = (int64_t)Hq * D; p.o_hs = D;
+  p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
+  p.causal = causal ? 1 : 0;
+  p.hdr = static_cast<WsHeader *>(workspace);
+  p.pairs = nullptr;
+  int sms = 0;
+  MXFA_TRY(sm_count(&sms));
+  DecodeSched s = decode_sched(p, Hkv, num_splits, D, kGqKeys, workspace, sms);
+  s.cache_seqlens = cache_seqlens;
+  s.add = Snew;
+  s.advance = Snew > 0 ? 1 : 0;
+  s.block_table = block_table;
+  s.max_blocks = paged ? max_blocks_per_seq : 0;
+  s.page_size = page_size;
+  const int64_t rows = (int64_t)num_pages * page_size;
+  if (Snew > 0) {
+    kv_append_kernel<<<dim3(Snew, batch), 256, 0, st>>>(p, s, k_new, v_new, Snew, (int)rows);
+    MXFA_CUDA(cudaGetLastError());
+  }
+  return launch_decode_gqa(p, s, dtype, rows, paged && page_size < kGqKeys ? page_size : kGqKeys, st);
 }
 
 }  // extern "C"

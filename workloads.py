@@ -181,6 +181,61 @@ def cfg_mla_decode() -> Problem:
     return mla_decode(3, 128, 4, 8192, name="mla_decode_b128_q4_h16_kv8192_bf16")
 
 
+def kvcache(seed: int, batch: int, Sq: int, Snew: int, seqlens: list[int], hq: int = 32, hkv: int = 4,
+            d: int = 128, dtype: str = "bf16", page_size: int | None = None, cache_len: int = 0,
+            causal: bool = False) -> dict:
+    """A KV-cache decode (mxflashattn flash_attn_with_kvcache): q [B, Sq, Hq, D],
+    a dense cache [B, cache_len, Hkv, D] (page_size None) or a paged one
+    [pages, page_size, Hkv, D] whose block table is a seeded permutation of
+    the pages, cache_seqlens, and rows k_new / v_new [B, Snew, Hkv, D].  Every
+    cache slot is filled with random values, so a key read past a sequence's
+    length shows up in the result.  Returns the device-independent tensors and
+    the equivalent packed Problem (keys in order, appended rows after the
+    cached ones) for the reference computation."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    lens = [L + Snew for L in seqlens]
+    q = _randn(g, (batch, Sq, hq, d), dtype)
+    k_new = _randn(g, (batch, Snew, hkv, d), dtype) if Snew else None
+    v_new = _randn(g, (batch, Snew, hkv, d), dtype) if Snew else None
+    if page_size is None:
+        cap = max(cache_len, max(lens))
+        kc = _randn(g, (batch, cap, hkv, d), dtype)
+        vc = _randn(g, (batch, cap, hkv, d), dtype)
+        table = None
+        rows = lambda b, pos: (b, pos)
+    else:
+        per = [(L + page_size - 1) // page_size for L in lens]
+        max_blocks = max(1, max(per))
+        pages = sum(per) + 3  # a few pages no sequence uses
+        kc = _randn(g, (pages, page_size, hkv, d), dtype)
+        vc = _randn(g, (pages, page_size, hkv, d), dtype)
+        perm = torch.randperm(pages, generator=g).tolist()
+        table = torch.full((batch, max_blocks), -1, dtype=torch.int32)
+        it = iter(perm)
+        for b in range(batch):
+            for i in range(per[b]):
+                table[b, i] = next(it)
+        rows = lambda b, pos: (int(table[b, pos // page_size]), pos % page_size)
+    # the logical keys of each entry after the append
+    ks, vs = [], []
+    for b in range(batch):
+        kb = torch.empty((lens[b], hkv, d), dtype=kc.dtype)
+        vb = torch.empty((lens[b], hkv, d), dtype=vc.dtype)
+        for pos in range(lens[b]):
+            if pos < seqlens[b]:
+                pg, off = rows(b, pos)
+                kb[pos], vb[pos] = kc[pg, off], vc[pg, off]
+            else:
+                kb[pos], vb[pos] = k_new[b, pos - seqlens[b]], v_new[b, pos - seqlens[b]]
+        ks.append(kb)
+        vs.append(vb)
+    prob = Problem(f"kvcache_b{batch}_sq{Sq}_new{Snew}", dtype, q.reshape(batch * Sq, hq, d), torch.cat(ks),
+                   torch.cat(vs), _cu([Sq] * batch), _cu(lens), hq, hkv, d, d, causal, d ** -0.5)
+    return {"q": q, "k_cache": kc, "v_cache": vc, "k_new": k_new, "v_new": v_new,
+            "cache_seqlens": torch.tensor(seqlens, dtype=torch.int32), "block_table": table, "rows": rows,
+            "lens": lens, "problem": prob}
+
+
 def cfg_gqa_decode(batch: int = 64, kv_len: int = 8192) -> Problem:
     """Grouped-query decode (next scope row): q_len 1, Hq 32, Hkv 4, D 128,
     bf16, kv_len 8192 per sequence, seed 6; KV 1.07 GB, larger than L2."""
