@@ -62,24 +62,32 @@ def decode_bytes(p):
     return kv + p.q.numel() * es + p.total_q * p.hq * p.dv * es + p.total_q * p.hq * 4
 
 
-def kernel_hash():
+# Source files that define each measured kernel (its own header and the
+# headers it includes); a recorded ncu capture is valid while they are unchanged.
+KERNEL_SOURCES = {
+    "attn_fwd_tc_kernel": ["prefill_tc.cuh", "exp2_poly.cuh", "ptx.cuh", "common.cuh"],
+    "decode": ["decode_tc.cuh", "ptx.cuh", "common.cuh"],
+    "decode_gqa": ["decode_gqa.cuh", "decode_tc.cuh", "ptx.cuh", "common.cuh"],
+}
+
+
+def kernel_hash(kernel: str):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "tiled_attention_21_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu capture, if it was taken on
-    the current kernel sources (else None)."""
+    the current sources of that kernel (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     d = json.load(open(path))
     e = d.get(kernel, {}).get(workload)
-    if not e or e.get("source_hash") != kernel_hash():
+    if not e or e.get("source_hash") != kernel_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
