@@ -41,6 +41,26 @@ def test_mla_ragged_lengths():
     check(p)
 
 
+def test_mla_one_long_sequence():
+    # 625 KV tiles of one sequence cut at every CTA boundary: every piece of
+    # the automatic schedule starts at a distinct cut inside the sequence
+    p = workloads.mla_decode(25, batch=1, q_len=4, kv_len=40000)
+    check(p)
+
+
+def test_mla_cuts_on_sequence_starts():
+    # 4 x 37 = 148 tiles of 64 keys over 148 CTAs: the cuts fall on every tile
+    # boundary, three of them on sequence starts (not cuts inside a sequence)
+    p = workloads.mla_decode(26, batch=4, q_len=4, kv_len=37 * 64)
+    check(p)
+
+
+def test_mla_fewer_tiles_than_ctas():
+    # 128 tiles for 148 CTAs: several cut values repeat (empty CTA ranges)
+    p = workloads.mla_decode(27, batch=1, q_len=4, kv_len=8192)
+    check(p)
+
+
 def test_mla_fp16_and_small_q():
     p = workloads.mla_decode(23, batch=4, q_len=1, kv_len=333, dtype="f16")
     check(p)

@@ -145,6 +145,7 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
   __shared__ typename Scan::TempStorage tmp;
   __shared__ int carry, max_n, split_mode;
   __shared__ int cut[kDcMaxGrid + 1];  // x_c = c*T/G, c = 0..G
+  __shared__ int ps[kDcMaxGrid + 1];   // ps[c]: c' in [1, c] with cut[c'] != cut[c'-1] (distinct cut values)
   const int tid = threadIdx.x, B = p.batch * s.heads, G = s.grid;
   if (tid == 0) {
     carry = 0;
@@ -182,7 +183,13 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     split_mode = (s.num_splits > 0) ? 1 : (5 * whole > 6 * even ? 2 : 0);  // 0 whole, 1 k pieces, 2 even cut
   }
   __syncthreads();
-  // first c with cut[c] > x (cut is non-decreasing)
+  {
+    int incl, total;
+    Scan(tmp).InclusiveSum((tid >= 1 && tid <= G && cut[tid] != cut[tid - 1]) ? 1 : 0, incl, total);
+    if (tid <= G) ps[tid] = incl;
+  }
+  __syncthreads();
+  // first c with cut[c] > x / with cut[c] >= x (cut is non-decreasing)
   auto upper = [&](int x) {
     int lo = 0, hi = G + 1;
     while (lo < hi) {
@@ -191,20 +198,24 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     }
     return lo;
   };
+  auto lower = [&](int x) {
+    int lo = 0, hi = G + 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (cut[mid] < x) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+  };
   auto pieces = [&](int b) -> int {
     const int n = s.n_tiles[b];
     if (n == 0) return 0;
     if (split_mode == 0) return 1;
     if (split_mode == 1) return min(s.num_splits, n);
-    // distinct cut values strictly inside (P, P + n)
+    // 1 + the distinct cut values strictly inside (P, P + n); the first cut
+    // above P always differs from the one before it
     const int P = s.tile_pre[b];
-    int cuts = 0, prev = P;
-    for (int c = upper(P); c < G && cut[c] < P + n; ++c)
-      if (cut[c] != prev) {
-        ++cuts;
-        prev = cut[c];
-      }
-    return 1 + cuts;
+    const int lo = upper(P), hi = lower(P + n);
+    return 1 + (hi > lo ? ps[hi - 1] - ps[lo - 1] : 0);
   };
   if (tid == 0) carry = 0;
   __syncthreads();
@@ -222,30 +233,43 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
   const int n_segs = carry;
   if (tid == 0) s.seg_base[B] = n_segs;
   __syncthreads();
+  // Segment list.  Each sequence writes its first piece (and, in modes 0
+  // and 1, all of them); in mode 2 every distinct cut value strictly inside
+  // a sequence writes the piece it starts, so no thread walks a long run of
+  // cuts.
   for (int b = tid; b < B; b += 1024) {
     const int n = s.n_tiles[b], P = s.tile_pre[b], k = s.seg_cnt[b];
-    int idx = s.seg_base[b];
+    const int idx = s.seg_base[b];
     if (k == 0) continue;
     if (split_mode == 1) {
       for (int i = 0; i < k; ++i) {
         const int t0 = (int)(((int64_t)i * n) / k), t1 = (int)(((int64_t)(i + 1) * n) / k);
-        if (idx < s.max_segs) s.segs[idx] = make_int4(b, t0, t1, P + t0);
-        ++idx;
+        if (idx + i < s.max_segs) s.segs[idx + i] = make_int4(b, t0, t1, P + t0);
       }
     } else {
-      int t0 = 0;
-      if (split_mode == 2) {
-        for (int c = upper(P); c < G && cut[c] < P + n; ++c) {
-          if (cut[c] > P + t0) {
-            if (idx < s.max_segs) s.segs[idx] = make_int4(b, t0, cut[c] - P, P + t0);
-            ++idx;
-            t0 = cut[c] - P;
-          }
-        }
-      }
-      if (idx < s.max_segs) s.segs[idx] = make_int4(b, t0, n, P + t0);
+      const int e0 = split_mode == 2 ? min(cut[upper(P)], P + n) : P + n;  // cut[G] = T > P
+      if (idx < s.max_segs) s.segs[idx] = make_int4(b, 0, e0 - P, P);
     }
   }
+  if (split_mode == 2) {
+    for (int c = 1 + tid; c < G; c += 1024) {
+      const int x = cut[c];
+      if (x == cut[c - 1] || x <= 0 || x >= T) continue;
+      // the sequence b with tile_pre[b] < x <= tile_pre[b + 1]
+      int lo = 1, hi = B;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (s.tile_pre[mid] < x) lo = mid + 1; else hi = mid;
+      }
+      const int b = lo - 1, P = s.tile_pre[b], n = s.n_tiles[b];
+      if (x >= P + n) continue;  // x starts the next sequence: not a cut inside b
+      const int k = ps[c] - ps[upper(P) - 1];  // this piece's index within b (>= 1)
+      const int e = min(cut[upper(x)], P + n);
+      const int idx = s.seg_base[b] + k;
+      if (idx < s.max_segs) s.segs[idx] = make_int4(b, x - P, e - P, x);
+    }
+  }
+  __syncthreads();
   if (tid == 0) {
     p.hdr->n_units = (uint32_t)min(n_segs, s.max_segs);
     p.hdr->n_aux = (uint32_t)T;
@@ -621,39 +645,81 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
 // v), DV/4 threads.  Row r of sequence v = (b, g) is query token r / G of
 // batch entry b, head g*G + r % G, with G = Hq / heads.
 template <typename T, int DV>
-__global__ void __launch_bounds__(DV / 4) decode_combine_kernel(const AttnParams p, const DecodeSched s) {
-  const int r = blockIdx.x, v = blockIdx.y;
-  const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
-  const int2 qr = dc_q(p, b);
-  const int q0 = qr.x, sq = qr.y;
-  if (r >= sq * G) return;
-  const int cnt = s.seg_cnt[v];
-  if (cnt == 1) return;  // stored directly by the decode kernel
-  const int tok = q0 + r / G, h = gh * G + r % G;
-  T *orow = reinterpret_cast<T *>(p.o) + (int64_t)tok * p.o_rs + (int64_t)h * p.o_hs;
-  const int base = s.seg_base[v];
-  float M = -INFINITY;
-  for (int i = 0; i < cnt; ++i) M = fmaxf(M, s.part_ml[(int64_t)(base + i) * kDcRows + r].x);
-  float L = 0.f;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (M != -INFINITY) {
-    for (int i = 0; i < cnt; ++i) {
-      const float2 ml = s.part_ml[(int64_t)(base + i) * kDcRows + r];
-      const float w = ex2(ml.x - M);  // 0 for a piece that saw no visible key
-      L += w * ml.y;
-      const float4 a = reinterpret_cast<const float4 *>(s.part_acc + ((int64_t)(base + i) * kDcRows + r) * DV)[threadIdx.x];
-      acc[0] = fmaf(w, a.x, acc[0]);
-      acc[1] = fmaf(w, a.y, acc[1]);
-      acc[2] = fmaf(w, a.z, acc[2]);
-      acc[3] = fmaf(w, a.w, acc[3]);
+__global__ void __launch_bounds__(DV) decode_combine_kernel(const AttnParams p, const DecodeSched s, int n_seq) {
+  // Grid-stride over items (sequence v, row r); an item whose sequence was
+  // not split (stored directly by the decode kernel) costs one load.  DV
+  // threads: four groups of DV/4; group q sums the pieces i = q, q+4, ...
+  // (each thread four columns), so four times as many partial loads are in
+  // flight, and the groups' sums are added in shared memory.
+  constexpr int kC = DV / 4;  // threads per group
+  __shared__ float red_m[DV];
+  __shared__ float4 red_acc[3][kC];
+  __shared__ float red_l[3];
+  const int grp = threadIdx.x / kC, col = threadIdx.x % kC;
+  const int n_items = n_seq * kDcRows;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int v = item / kDcRows, r = item % kDcRows;
+    const int cnt = s.seg_cnt[v];
+    // not split: stored directly by the decode kernel (a sequence with no
+    // piece, cnt = 0, is written here: O = 0, LSE = -inf)
+    if (cnt == 1) continue;
+    const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
+    const int2 qr = dc_q(p, b);
+    if (r >= qr.y * G) continue;
+    const int tok = qr.x + r / G, h = gh * G + r % G;
+    T *orow = reinterpret_cast<T *>(p.o) + (int64_t)tok * p.o_rs + (int64_t)h * p.o_hs;
+    const int base = s.seg_base[v];
+    // M = the largest piece maximum (all threads take part)
+    float m = -INFINITY;
+    for (int i = threadIdx.x; i < cnt; i += DV) m = fmaxf(m, s.part_ml[(int64_t)(base + i) * kDcRows + r].x);
+    red_m[threadIdx.x] = m;
+    __syncthreads();
+    for (int w = DV / 2; w > 0; w >>= 1) {
+      if (threadIdx.x < w) red_m[threadIdx.x] = fmaxf(red_m[threadIdx.x], red_m[threadIdx.x + w]);
+      __syncthreads();
     }
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  const int d = threadIdx.x * 4;
+    const float M = red_m[0];
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+#pragma unroll 4
+      for (int i = grp; i < cnt; i += 4) {
+        const float2 ml = s.part_ml[(int64_t)(base + i) * kDcRows + r];
+        const float w = ex2(ml.x - M);  // 0 for a piece that saw no visible key
+        L += w * ml.y;
+        const float4 a = reinterpret_cast<const float4 *>(s.part_acc + ((int64_t)(base + i) * kDcRows + r) * DV)[col];
+        acc.x = fmaf(w, a.x, acc.x);
+        acc.y = fmaf(w, a.y, acc.y);
+        acc.z = fmaf(w, a.z, acc.z);
+        acc.w = fmaf(w, a.w, acc.w);
+      }
+    }
+    if (grp > 0) {
+      red_acc[grp - 1][col] = acc;
+      if (col == 0) red_l[grp - 1] = L;
+    }
+    __syncthreads();
+    if (grp == 0) {
 #pragma unroll
-  for (int e = 0; e < 4; ++e) orow[d + e] = from_f32<T>(acc[e] * inv);
-  if (threadIdx.x == 0 && p.lse)
-    p.lse[(int64_t)tok * p.hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
+      for (int q = 0; q < 3; ++q) {
+        const float4 o = red_acc[q][col];
+        acc.x += o.x;
+        acc.y += o.y;
+        acc.z += o.z;
+        acc.w += o.w;
+        L += red_l[q];
+      }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const int d = col * 4;
+      orow[d + 0] = from_f32<T>(acc.x * inv);
+      orow[d + 1] = from_f32<T>(acc.y * inv);
+      orow[d + 2] = from_f32<T>(acc.z * inv);
+      orow[d + 3] = from_f32<T>(acc.w * inv);
+      if (col == 0 && p.lse)
+        p.lse[(int64_t)tok * p.hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
+    }
+    __syncthreads();  // red_m / red_acc are reused by the next item
+  }
 }
 
 }  // namespace mxfa

@@ -367,6 +367,13 @@ DecodeSched decode_sched(const AttnParams &p, int heads, int num_splits, int dv,
 
 // `kv_rows`: rows of the K / V tensors; `box`: TMA box height (128, or the
 // page size of a paged cache with pages shorter than a tile).
+// Blocks of the combine kernel: it walks (sequence, row) items with a grid
+// stride, two blocks per SM of the decode grid at most.
+int combine_grid(int n_seq, int decode_grid) {
+  const int64_t items = (int64_t)n_seq * kDcRows;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(items, 2 * (int64_t)decode_grid));
+}
+
 template <int D, bool BF16>
 mxfa_status_t launch_decode_gqa_t(AttnParams &p, const DecodeSched &s, mxfa_dtype_t dt, int64_t kv_rows, int box,
                                   cudaStream_t st) {
@@ -380,7 +387,8 @@ mxfa_status_t launch_decode_gqa_t(AttnParams &p, const DecodeSched &s, mxfa_dtyp
   k<<<s.grid, kGqThreads, GqaCfg<D>::kSmemBytes, st>>>(p, s, mk, mv);
   MXFA_CUDA(cudaGetLastError());
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  decode_combine_kernel<T, D><<<dim3(kDcRows, p.batch * p.hkv), D / 4, 0, st>>>(p, s);
+  const int n_seq = p.batch * p.hkv;
+  decode_combine_kernel<T, D><<<combine_grid(n_seq, s.grid), D, 0, st>>>(p, s, n_seq);
   MXFA_CUDA(cudaGetLastError());
   return MXFA_OK;
 }
@@ -409,12 +417,12 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
     MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(attn_decode_tc_kernel<true>), kDcSmemBytes));
     attn_decode_tc_kernel<true><<<s.grid, kDcThreads, kDcSmemBytes, st>>>(p, s, mq, mkv);
     MXFA_CUDA(cudaGetLastError());
-    decode_combine_kernel<__nv_bfloat16, kDcDv><<<dim3(kDcRows, p.batch), kDcDv / 4, 0, st>>>(p, s);
+    decode_combine_kernel<__nv_bfloat16, kDcDv><<<combine_grid(p.batch, s.grid), kDcDv, 0, st>>>(p, s, p.batch);
   } else {
     MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(attn_decode_tc_kernel<false>), kDcSmemBytes));
     attn_decode_tc_kernel<false><<<s.grid, kDcThreads, kDcSmemBytes, st>>>(p, s, mq, mkv);
     MXFA_CUDA(cudaGetLastError());
-    decode_combine_kernel<__half, kDcDv><<<dim3(kDcRows, p.batch), kDcDv / 4, 0, st>>>(p, s);
+    decode_combine_kernel<__half, kDcDv><<<combine_grid(p.batch, s.grid), kDcDv, 0, st>>>(p, s, p.batch);
   }
   MXFA_CUDA(cudaGetLastError());
   return MXFA_OK;
