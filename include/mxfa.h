@@ -163,6 +163,14 @@ mxfa_status_t mxfa_attn_varlen_fwd_noalloc(const void *q, const void *k, const v
  * num_splits: 0 = automatic (the KV of all sequences is cut into
  *   near-equal pieces, one run per SM); k >= 1 = every sequence's KV is cut
  *   into k pieces.  The result does not depend on it beyond fp32 rounding.
+ * Small problems (the MLA-shaped kernel, num_splits = 0, batch no larger
+ *   than the SM count and batch * ceil(max_kv_len / 64) at most four tiles per
+ *   SM) run as one cooperative kernel launch, preceded by a small memset of
+ *   per-sequence counters in the workspace.  Each sequence is cut into
+ *   near-equal pieces, one CTA each, and the pieces of a sequence merge their
+ *   partials in the same kernel, so no schedule or combine kernel runs.  This
+ *   is the launch-bound regime for which the MLA decode page switches to a
+ *   different kernel (q_len * kv_len <= 4096).
  */
 size_t mxfa_attn_decode_splitkv_workspace_size(int batch, int max_q_len, int Hq, int Hkv, int Dv, int max_kv_len,
                                                int num_splits, mxfa_dtype_t dtype);

@@ -61,6 +61,22 @@ def test_mla_fewer_tiles_than_ctas():
     check(p)
 
 
+def test_mla_empty_sequences_single_launch():
+    # a small problem (one-launch schedule) with sequences that have no key
+    p = workloads.mla_decode(28, batch=4, q_len=4, kv_len=0, lens_kv=[0, 100, 0, 700])
+    check(p)
+
+
+def test_mla_single_launch_matches_split_schedule():
+    # the same small problem through the one-launch schedule (automatic) and
+    # through the prep + decode + combine schedule (fixed split count)
+    p = workloads.mla_decode(29, batch=2, q_len=4, kv_len=3000)
+    _, (o0, l0) = check(p, 0)
+    _, (o5, l5) = check(p, 5)
+    assert (o0.float() - o5.float()).abs().max() <= 4e-3
+    assert (l0 - l5).abs().max() <= 1e-4
+
+
 def test_mla_fp16_and_small_q():
     p = workloads.mla_decode(23, batch=4, q_len=1, kv_len=333, dtype="f16")
     check(p)

@@ -82,6 +82,13 @@ struct DecodeSched {
   int *kv_len;
   const int32_t *block_table;
   int max_blocks, page_size;
+  // Single-launch schedule (arith_k > 0, packed kv_indptr only): sequence v
+  // is cut into k_v = min(arith_k, its KV tiles) near-equal pieces and piece
+  // i is CTA v*arith_k + i, so no prep kernel runs.  The pieces of a split
+  // sequence merge their partials at the end of the same kernel; sync[v]
+  // counts the pieces that have stored theirs (zeroed before the launch).
+  int arith_k;
+  int *sync;
 };
 
 // Queries of batch entry b: (first row, count); packed (cu_q) or uniform.
@@ -116,10 +123,29 @@ struct DecodeCtrl {
 
 enum : uint32_t {
   kDSiteSlotEmpty = 0x301, kDSiteQReady, kDSiteSlotFull, kDSitePFull, kDSiteOEmpty, kDSiteSFull,
-  kDSiteODone, kDSiteSFree
+  kDSiteODone, kDSiteSFree, kDSiteMerge
 };
 
 __device__ __forceinline__ int dc_range_start(int c, int T, int G) { return (int)(((int64_t)c * T) / G); }
+
+// KV tiles of decode sequence v (0 when its batch entry has no query).
+__device__ __forceinline__ int dc_seq_tiles(const AttnParams &p, const DecodeSched &s, int v) {
+  const int b = v / s.heads;
+  if (dc_q(p, b).y <= 0) return 0;
+  return (dc_klen(p, s, b) + s.keys - 1) / s.keys;
+}
+// Pieces of sequence v.
+__device__ __forceinline__ int dc_seg_cnt(const AttnParams &p, const DecodeSched &s, int v) {
+  return s.arith_k > 0 ? min(s.arith_k, dc_seq_tiles(p, s, v)) : s.seg_cnt[v];
+}
+// Piece sg: (sequence, first tile, end tile, global first tile; the last
+// is not used by the single-launch schedule).
+__device__ __forceinline__ int4 dc_seg(const AttnParams &p, const DecodeSched &s, int sg) {
+  if (s.arith_k == 0) return s.segs[sg];
+  const int v = sg / s.arith_k, i = sg % s.arith_k;
+  const int n = dc_seq_tiles(p, s, v), k = max(1, min(s.arith_k, n));
+  return make_int4(v, (int)(((int64_t)i * n) / k), (int)(((int64_t)(i + 1) * n) / k), 0);
+}
 
 // First segment whose first global tile is >= x.
 __device__ __forceinline__ int dc_lower_bound(const int4 *segs, int n, int x) {
@@ -278,6 +304,121 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
 }
 
 // ----------------------------------------------------------------------------
+// Single-launch schedule: merge of a split sequence at the end of the decode
+// kernel.  Piece i of the k pieces of sequence v, once its partial is
+// stored, announces it on s.sync[v] and waits (bounded) until all k have;
+// it then merges slice i of the sequence's (row, 4-column) outputs with the
+// weights 2^(m_t - M) of decode_combine_kernel.  The pieces of a sequence
+// run at the same time (the kernel is launched cooperatively, one CTA per
+// piece).  Every thread of the CTA calls it; `scratch` is shared memory no
+// longer in use, at least 192 + rows + 2k floats.
+template <int NT>
+__device__ __forceinline__ float dc_block_reduce(float x, bool is_max, float *red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float y = __shfl_xor_sync(0xffffffffu, x, o);
+    x = is_max ? fmaxf(x, y) : x + y;
+  }
+  if (lane == 0) red[warp] = x;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < NT / 32; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  __syncthreads();  // red is reused
+  return r;
+}
+
+template <typename T, int DV, int NT>
+__device__ void dc_merge_pieces(const AttnParams &p, const DecodeSched &s, int v, int i, int k, float *scratch) {
+  volatile int *flag = reinterpret_cast<volatile int *>(scratch);
+  float *red = scratch + 32, *Mr = scratch + 64, *Lr = scratch + 128, *w = scratch + 192;
+  __threadfence();  // this thread's partial stores are visible to the other pieces
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    atomicAdd(s.sync + v, 1);
+    const uint64_t t0 = global_ns();
+    int good = 1;
+    while (*reinterpret_cast<volatile int *>(s.sync + v) < k) {
+      if (global_ns() - t0 > kWaitBudgetNs) {
+        report_error(p.hdr, kStatusTimeout, kDSiteMerge);
+        good = 0;
+        break;
+      }
+    }
+    *flag = good;
+  }
+  __syncthreads();
+  if (!*flag) return;
+  __threadfence();
+  const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
+  const int2 qr = dc_q(p, b);
+  const int rows = qr.y * G;
+  constexpr int C4 = DV / 4;
+  const int n_items = rows * C4;
+  const int lo = (int)(((int64_t)i * n_items) / k), hi = (int)(((int64_t)(i + 1) * n_items) / k);
+  if (lo >= hi) return;
+  const int r_lo = lo / C4, r_hi = (hi - 1) / C4 + 1;
+  const int base = v * s.arith_k;  // partial slot of piece 0
+  for (int r = r_lo; r < r_hi; ++r) {
+    float m = -INFINITY;
+    for (int t = threadIdx.x; t < k; t += NT) m = fmaxf(m, s.part_ml[(int64_t)(base + t) * kDcRows + r].x);
+    const float M = dc_block_reduce<NT>(m, true, red);
+    float ls = 0.f;
+    for (int t = threadIdx.x; t < k; t += NT) {
+      const float2 ml = s.part_ml[(int64_t)(base + t) * kDcRows + r];
+      const float wt = M == -INFINITY ? 0.f : ex2(ml.x - M);  // 0 for a piece that saw no visible key
+      w[(r - r_lo) * k + t] = wt;
+      ls += wt * ml.y;
+    }
+    const float L = dc_block_reduce<NT>(ls, false, red);
+    if (threadIdx.x == 0) {
+      Mr[r - r_lo] = M;
+      Lr[r - r_lo] = L;
+    }
+  }
+  __syncthreads();
+  for (int it = lo + threadIdx.x; it < hi; it += NT) {
+    const int r = it / C4, c4 = it % C4;
+    const float *wr = w + (r - r_lo) * k;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int t = 0; t < k; ++t) {
+      const float wt = wr[t];
+      const float4 a = reinterpret_cast<const float4 *>(s.part_acc + ((int64_t)(base + t) * kDcRows + r) * DV)[c4];
+      acc.x = fmaf(wt, a.x, acc.x);
+      acc.y = fmaf(wt, a.y, acc.y);
+      acc.z = fmaf(wt, a.z, acc.z);
+      acc.w = fmaf(wt, a.w, acc.w);
+    }
+    const float L = Lr[r - r_lo], inv = L > 0.f ? 1.f / L : 0.f;
+    const int tok = qr.x + r / G, h = gh * G + r % G;
+    T *orow = reinterpret_cast<T *>(p.o) + (int64_t)tok * p.o_rs + (int64_t)h * p.o_hs + 4 * c4;
+    orow[0] = from_f32<T>(acc.x * inv);
+    orow[1] = from_f32<T>(acc.y * inv);
+    orow[2] = from_f32<T>(acc.z * inv);
+    orow[3] = from_f32<T>(acc.w * inv);
+    if (c4 == 0 && p.lse)
+      p.lse[(int64_t)tok * p.hq + h] = L > 0.f ? (Mr[r - r_lo] + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
+  }
+}
+
+// Single-launch schedule: a sequence with no piece (no key, or no query)
+// gets O = 0 and LSE = -inf, written by its CTA 0.
+template <typename T, int DV, int NT>
+__device__ void dc_zero_rows(const AttnParams &p, const DecodeSched &s, int v) {
+  const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
+  const int2 qr = dc_q(p, b);
+  const int rows = qr.y * G;
+  for (int it = threadIdx.x; it < rows * DV; it += NT) {
+    const int r = it / DV, c = it % DV;
+    const int tok = qr.x + r / G, h = gh * G + r % G;
+    reinterpret_cast<T *>(p.o)[(int64_t)tok * p.o_rs + (int64_t)h * p.o_hs + c] = from_f32<T>(0.f);
+    if (c == 0 && p.lse) p.lse[(int64_t)tok * p.hq + h] = -INFINITY;
+  }
+}
+
+// ----------------------------------------------------------------------------
 template <bool BF16>
 __global__ void __launch_bounds__(kDcThreads, 1)
 attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
@@ -322,11 +463,18 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
 
-  // This CTA's pieces: those whose first tile lies in its tile range.
-  const int n_segs = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_units);
-  const int T = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_aux);
-  const int seg_lo = dc_lower_bound(s.segs, n_segs, dc_range_start(blockIdx.x, T, gridDim.x));
-  const int seg_hi = dc_lower_bound(s.segs, n_segs, dc_range_start(blockIdx.x + 1, T, gridDim.x));
+  // This CTA's pieces: those whose first tile lies in its tile range (or,
+  // in the single-launch schedule, piece blockIdx.x if it exists).
+  int seg_lo, seg_hi;
+  if (s.arith_k > 0) {
+    seg_lo = blockIdx.x;
+    seg_hi = (int)(blockIdx.x % s.arith_k) < dc_seg_cnt(p, s, blockIdx.x / s.arith_k) ? seg_lo + 1 : seg_lo;
+  } else {
+    const int n_segs = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_units);
+    const int T = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_aux);
+    seg_lo = dc_lower_bound(s.segs, n_segs, dc_range_start(blockIdx.x, T, gridDim.x));
+    seg_hi = dc_lower_bound(s.segs, n_segs, dc_range_start(blockIdx.x + 1, T, gridDim.x));
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -334,10 +482,10 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       uint32_t tc = 0;  // tiles issued by this CTA
       bool ok = true;
       for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
-        const int4 sd = s.segs[sg];
+        const int4 sd = dc_seg(p, s, sg);
         const int k0 = p.cu_k[sd.x];
         if (sg + 1 < seg_hi) {  // the next piece's query rows, into L2
-          const int bn = s.segs[sg + 1].x;
+          const int bn = dc_seg(p, s, sg + 1).x;
           const int64_t q0n = p.cu_q[bn], rn = (p.cu_q[bn + 1] - q0n) * p.hq;
           if (rn > 0)
             tma_prefetch_bytes(reinterpret_cast<const uint16_t *>(p.q) + q0n * p.hq * kDcDqk,
@@ -403,7 +551,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         return true;
       };
       for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
-        const int4 sd = s.segs[sg];
+        const int4 sd = dc_seg(p, s, sg);
         const int n = sd.z - sd.y;
         if (!wait_warp(b_qr, (sg - seg_lo) & 1, abort_flag, hdr, kDSiteQReady)) break;
         tc_fence_after();
@@ -455,7 +603,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     // Q rows of piece sg into TMEM (lanes 16-31, columns kDcQCol..): this
     // thread writes half `half` of row r; all global loads are issued first.
     auto load_q = [&](int sg) {
-      const int bq = s.segs[sg].x;
+      const int bq = dc_seg(p, s, sg).x;
       const int q0 = p.cu_q[bq], rows = (p.cu_q[bq + 1] - q0) * p.hq;
       const uint4 *src = reinterpret_cast<const uint4 *>(
           reinterpret_cast<const uint16_t *>(p.q) + ((int64_t)q0 * p.hq + r) * kDcDqk);
@@ -492,7 +640,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     bool ok = true;
     if (seg_lo < seg_hi) load_q(seg_lo);
     for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
-      const int4 sd = s.segs[sg];
+      const int4 sd = dc_seg(p, s, sg);
       const int b = sd.x;
       const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0, sk = p.cu_k[b + 1] - p.cu_k[b];
       const int rows = sq * p.hq;
@@ -592,7 +740,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         if (!__all_sync(0xffffffffu, got_o)) break;
         tc_fence_after();
       }
-      const bool direct = s.seg_cnt[b] == 1;
+      const bool direct = dc_seg_cnt(p, s, b) == 1;
       const int tok = q0 + (valid ? r / p.hq : 0), h = valid ? r % p.hq : 0;
       using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -637,6 +785,15 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+  if (s.arith_k > 0) {
+    // single-launch schedule: the pieces of a split sequence merge here (the
+    // KV ring, drained above, is the scratch space)
+    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    const int v = blockIdx.x / s.arith_k, i = blockIdx.x % s.arith_k, k = dc_seg_cnt(p, s, v);
+    float *scratch = reinterpret_cast<float *>(smem_raw + kDcCtrlBytes);
+    if (k > 1 && i < k) dc_merge_pieces<T, kDcDv, kDcThreads>(p, s, v, i, k, scratch);
+    else if (k == 0 && i == 0) dc_zero_rows<T, kDcDv, kDcThreads>(p, s, v);
   }
 }
 

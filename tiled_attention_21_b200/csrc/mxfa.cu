@@ -307,7 +307,7 @@ mxfa_status_t prefill(AttnParams &p, mxfa_dtype_t dt, int D, bool varlen, int64_
 // sequences (batch entries x KV heads that form separate sequences), Dv
 // output columns.
 struct DecodeWs {
-  size_t n_tiles, tile_pre, seg_base, seg_cnt, kv_len, segs, part_ml, part_acc, total;
+  size_t n_tiles, tile_pre, seg_base, seg_cnt, kv_len, sync, segs, part_ml, part_acc, total;
   int max_segs;
 };
 DecodeWs decode_ws(int batch, int max_kv_len, int num_splits, int dv, int keys) {
@@ -319,7 +319,8 @@ DecodeWs decode_ws(int batch, int max_kv_len, int num_splits, int dv, int keys) 
   w.seg_base = w.tile_pre + align256(sizeof(int) * (size_t)(batch + 1));
   w.seg_cnt = w.seg_base + align256(sizeof(int) * (size_t)(batch + 1));
   w.kv_len = w.seg_cnt + align256(sizeof(int) * (size_t)batch);
-  w.segs = w.kv_len + align256(sizeof(int) * (size_t)batch);
+  w.sync = w.kv_len + align256(sizeof(int) * (size_t)batch);
+  w.segs = w.sync + align256(sizeof(int) * (size_t)batch);
   w.part_ml = w.segs + align256(sizeof(int4) * (size_t)w.max_segs);
   w.part_acc = w.part_ml + align256(sizeof(float2) * (size_t)w.max_segs * kDcRows);
   w.total = w.part_acc + align256(sizeof(float) * (size_t)w.max_segs * kDcRows * dv);
@@ -355,6 +356,8 @@ DecodeSched decode_sched(const AttnParams &p, int heads, int num_splits, int dv,
   s.part_ml = reinterpret_cast<float2 *>(base + w.part_ml);
   s.part_acc = reinterpret_cast<float *>(base + w.part_acc);
   s.kv_len = reinterpret_cast<int *>(base + w.kv_len);
+  s.sync = reinterpret_cast<int *>(base + w.sync);
+  s.arith_k = 0;
   s.max_segs = w.max_segs;
   s.num_splits = num_splits;
   s.grid = std::min(sms, kDcMaxGrid);
@@ -411,6 +414,21 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
   CUtensorMap mq, mkv;
   MXFA_TRY(make_map_2d(&mq, p.q, dt, kDcDqk, (int64_t)total_q * p.hq, kDcDqk));
   MXFA_TRY(make_map_2d(&mkv, p.k, dt, kDcDqk, total_kv, p.k_rs));
+  // Small problems run in one launch: no prep kernel (the pieces follow from
+  // kv_indptr) and no combine kernel (split sequences merge in the kernel).
+  const int max_tiles = (p.max_sk + kDcKeys - 1) / kDcKeys;
+  if (num_splits == 0 && p.batch <= s.grid && (int64_t)p.batch * max_tiles <= 4 * (int64_t)s.grid) {
+    DecodeSched sa = s;
+    const int t_min = max_tiles > 32 ? 4 : 2;  // tiles per piece at least (merge cost vs chain length)
+    sa.arith_k = std::max(1, std::min(s.grid / p.batch, (max_tiles + t_min - 1) / t_min));
+    if (sa.arith_k > 1) MXFA_CUDA(cudaMemsetAsync(sa.sync, 0, sizeof(int) * (size_t)p.batch, st));
+    const void *k = dt == MXFA_BF16 ? reinterpret_cast<const void *>(attn_decode_tc_kernel<true>)
+                                    : reinterpret_cast<const void *>(attn_decode_tc_kernel<false>);
+    MXFA_TRY(ensure_smem(k, kDcSmemBytes));
+    void *args[] = {&p, &sa, &mq, &mkv};
+    MXFA_CUDA(cudaLaunchCooperativeKernel(k, dim3(p.batch * sa.arith_k), dim3(kDcThreads), args, kDcSmemBytes, st));
+    return MXFA_OK;
+  }
   decode_prep_kernel<<<1, 1024, 0, st>>>(p, s);
   MXFA_CUDA(cudaGetLastError());
   if (dt == MXFA_BF16) {
