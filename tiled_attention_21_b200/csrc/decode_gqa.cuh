@@ -103,11 +103,18 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
 
-  // This CTA's pieces: those whose first tile lies in its tile range.
-  const int n_segs = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_units);
-  const int T = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_aux);
-  const int seg_lo = dc_lower_bound(s.segs, n_segs, dc_range_start(blockIdx.x, T, gridDim.x));
-  const int seg_hi = dc_lower_bound(s.segs, n_segs, dc_range_start(blockIdx.x + 1, T, gridDim.x));
+  // This CTA's pieces: those whose first tile lies in its tile range (or,
+  // in the single-launch schedule, piece blockIdx.x if it exists).
+  int seg_lo, seg_hi;
+  if (s.arith_k > 0) {
+    seg_lo = blockIdx.x;
+    seg_hi = (int)(blockIdx.x % s.arith_k) < dc_seg_cnt(p, s, blockIdx.x / s.arith_k) ? seg_lo + 1 : seg_lo;
+  } else {
+    const int n_segs = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_units);
+    const int T = (int)*reinterpret_cast<volatile uint32_t *>(&hdr->n_aux);
+    seg_lo = dc_lower_bound(s.segs, n_segs, dc_range_start(blockIdx.x, T, gridDim.x));
+    seg_hi = dc_lower_bound(s.segs, n_segs, dc_range_start(blockIdx.x + 1, T, gridDim.x));
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -115,7 +122,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
       uint32_t tc = 0;  // tiles issued by this CTA
       bool ok = true;
       for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
-        const int4 sd = s.segs[sg];
+        const int4 sd = dc_seg(p, s, sg);
         const int b = sd.x / s.heads, g = sd.x % s.heads;
         const int len = dc_klen(p, s, b);
         for (int j = sd.y; ok && j < sd.z; ++j, ++tc) {
@@ -187,7 +194,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
       return true;
     };
     for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
-      const int4 sd = s.segs[sg];
+      const int4 sd = dc_seg(p, s, sg);
       const int n = sd.z - sd.y;
       if (!wait_warp(b_qr, (sg - seg_lo) & 1, kDSiteQReady)) break;
       tc_fence_after();
@@ -240,7 +247,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     // Q rows of piece sg into TMEM (lanes 16-31, columns kGqQCol..): this
     // thread writes half `half` of row r.
     auto load_q = [&](int sg) {
-      const int v = s.segs[sg].x, b = v / s.heads, gh = v % s.heads;
+      const int v = dc_seg(p, s, sg).x, b = v / s.heads, gh = v % s.heads;
       const int q0 = dc_q(p, b).x, rows = dc_q(p, b).y * G;
       const bool vq = r < rows;
       const uint4 *src = reinterpret_cast<const uint4 *>(
@@ -262,7 +269,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     bool ok = true;
     if (seg_lo < seg_hi) load_q(seg_lo);
     for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
-      const int4 sd = s.segs[sg];
+      const int4 sd = dc_seg(p, s, sg);
       const int v = sd.x, b = v / s.heads, gh = v % s.heads;
       const int q0 = dc_q(p, b).x, sq = dc_q(p, b).y, sk = dc_klen(p, s, b);
       const int rows = sq * G;
@@ -375,7 +382,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
         if (!__all_sync(0xffffffffu, got_o)) break;
         tc_fence_after();
       }
-      const bool direct = s.seg_cnt[v] == 1;
+      const bool direct = dc_seg_cnt(p, s, v) == 1;
       const int tok = q0 + (valid ? r / G : 0), h = gh * G + (valid ? r % G : 0);
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
@@ -419,6 +426,15 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+  if (s.arith_k > 0) {
+    // single-launch schedule: the pieces of a split sequence merge here (the
+    // K/V ring, drained above, is the scratch space)
+    using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+    const int v = blockIdx.x / s.arith_k, i = blockIdx.x % s.arith_k, k = dc_seg_cnt(p, s, v);
+    float *scratch = reinterpret_cast<float *>(smem_raw + kDcCtrlBytes);
+    if (k > 1 && i < k) dc_merge_pieces<T, D, kGqThreads>(p, s, v, i, k, scratch);
+    else if (k == 0 && i == 0) dc_zero_rows<T, D, kGqThreads>(p, s, v);
   }
 }
 

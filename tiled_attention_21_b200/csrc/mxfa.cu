@@ -383,14 +383,26 @@ mxfa_status_t launch_decode_gqa_t(AttnParams &p, const DecodeSched &s, mxfa_dtyp
   CUtensorMap mk, mv;
   MXFA_TRY(make_map(&mk, p.k, dt, D, p.hkv, kv_rows, p.k_rs, p.k_hs, box));
   MXFA_TRY(make_map(&mv, p.v, dt, D, p.hkv, kv_rows, p.v_rs, p.v_hs, box));
+  auto k = attn_decode_gqa_kernel<D, BF16>;
+  // Small problems on packed K/V run in one launch, as for the MLA kernel.
+  const int n_seq = p.batch * p.hkv, max_tiles = (p.max_sk + kGqKeys - 1) / kGqKeys;
+  if (s.num_splits == 0 && p.cu_k && n_seq <= s.grid && (int64_t)n_seq * max_tiles <= 4 * (int64_t)s.grid) {
+    DecodeSched sa = s;
+    const int t_min = max_tiles > 16 ? 4 : 2;  // tiles per piece at least (merge cost vs chain length)
+    sa.arith_k = std::max(1, std::min(s.grid / n_seq, (max_tiles + t_min - 1) / t_min));
+    if (sa.arith_k > 1) MXFA_CUDA(cudaMemsetAsync(sa.sync, 0, sizeof(int) * (size_t)n_seq, st));
+    MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(k), GqaCfg<D>::kSmemBytes));
+    void *args[] = {&p, &sa, &mk, &mv};
+    MXFA_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(k), dim3(n_seq * sa.arith_k),
+                                          dim3(kGqThreads), args, GqaCfg<D>::kSmemBytes, st));
+    return MXFA_OK;
+  }
   decode_prep_kernel<<<1, 1024, 0, st>>>(p, s);
   MXFA_CUDA(cudaGetLastError());
-  auto k = attn_decode_gqa_kernel<D, BF16>;
   MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(k), GqaCfg<D>::kSmemBytes));
   k<<<s.grid, kGqThreads, GqaCfg<D>::kSmemBytes, st>>>(p, s, mk, mv);
   MXFA_CUDA(cudaGetLastError());
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  const int n_seq = p.batch * p.hkv;
   decode_combine_kernel<T, D><<<combine_grid(n_seq, s.grid), D, 0, st>>>(p, s, n_seq);
   MXFA_CUDA(cudaGetLastError());
   return MXFA_OK;
