@@ -402,10 +402,9 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
           for (int e = 0; e < 4; ++e)
             reinterpret_cast<uint4 *>(orow)[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         } else {
-          float4 *dst = reinterpret_cast<float4 *>(s.part_acc + ((int64_t)sg * kDcRows + r) * D + col);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
+            *dc_pacc<D>(s, sg, r, col / 4 + e) = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
                                  __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
         }
       }

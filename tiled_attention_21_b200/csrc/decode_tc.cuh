@@ -128,6 +128,28 @@ enum : uint32_t {
 
 __device__ __forceinline__ int dc_range_start(int c, int T, int G) { return (int)(((int64_t)c * T) / G); }
 
+// Four outputs, rounded to the 16-bit output type, as one 8-byte store.
+template <typename T>
+__device__ __forceinline__ void dc_store4(T *dst, float a, float b, float c, float d) {
+  uint32_t lo, hi;
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    lo = pack_bf16x2(a, b);
+    hi = pack_bf16x2(c, d);
+  } else {
+    lo = pack_f16x2(a, b);
+    hi = pack_f16x2(c, d);
+  }
+  *reinterpret_cast<uint2 *>(dst) = make_uint2(lo, hi);
+}
+
+// Partial accumulator of piece sg, row r, columns 4*c4 .. 4*c4+3: layout
+// [piece][DV/4][64 rows] in float4 units, so the threads that hold
+// consecutive rows of the same four columns touch consecutive 16-byte words.
+template <int DV>
+__device__ __forceinline__ float4 *dc_pacc(const DecodeSched &s, int sg, int r, int c4) {
+  return reinterpret_cast<float4 *>(s.part_acc) + ((int64_t)sg * (DV / 4) + c4) * kDcRows + r;
+}
+
 // KV tiles of decode sequence v (0 when its batch entry has no query).
 __device__ __forceinline__ int dc_seq_tiles(const AttnParams &p, const DecodeSched &s, int v) {
   const int b = v / s.heads;
@@ -311,28 +333,16 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
 // weights 2^(m_t - M) of decode_combine_kernel.  The pieces of a sequence
 // run at the same time (the kernel is launched cooperatively, one CTA per
 // piece).  Every thread of the CTA calls it; `scratch` is shared memory no
-// longer in use, at least 192 + rows + 2k floats.
-template <int NT>
-__device__ __forceinline__ float dc_block_reduce(float x, bool is_max, float *red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float y = __shfl_xor_sync(0xffffffffu, x, o);
-    x = is_max ? fmaxf(x, y) : x + y;
-  }
-  if (lane == 0) red[warp] = x;
-  __syncthreads();
-  float r = red[0];
-#pragma unroll
-  for (int w = 1; w < NT / 32; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
-  __syncthreads();  // red is reused
-  return r;
-}
-
+// longer in use, 160 + 128 k floats.
 template <typename T, int DV, int NT>
 __device__ void dc_merge_pieces(const AttnParams &p, const DecodeSched &s, int v, int i, int k, float *scratch) {
   volatile int *flag = reinterpret_cast<volatile int *>(scratch);
-  float *red = scratch + 32, *Mr = scratch + 64, *Lr = scratch + 128, *w = scratch + 192;
+  const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
+  const int2 qr = dc_q(p, b);
+  const int rows = qr.y * G;
+  // scratch: flag, then per row M and L, then the weights w and sums l of
+  // every (row, piece)
+  float *Mr = scratch + 32, *Lr = Mr + kDcRows, *w = Lr + kDcRows, *wl = w + rows * k;
   __threadfence();  // this thread's partial stores are visible to the other pieces
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -351,55 +361,78 @@ __device__ void dc_merge_pieces(const AttnParams &p, const DecodeSched &s, int v
   __syncthreads();
   if (!*flag) return;
   __threadfence();
-  const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
-  const int2 qr = dc_q(p, b);
-  const int rows = qr.y * G;
   constexpr int C4 = DV / 4;
+  // This piece's slice of the (4-column group, row) items, rows fastest.
   const int n_items = rows * C4;
   const int lo = (int)(((int64_t)i * n_items) / k), hi = (int)(((int64_t)(i + 1) * n_items) / k);
   if (lo >= hi) return;
-  const int r_lo = lo / C4, r_hi = (hi - 1) / C4 + 1;
   const int base = v * s.arith_k;  // partial slot of piece 0
-  for (int r = r_lo; r < r_hi; ++r) {
-    float m = -INFINITY;
-    for (int t = threadIdx.x; t < k; t += NT) m = fmaxf(m, s.part_ml[(int64_t)(base + t) * kDcRows + r].x);
-    const float M = dc_block_reduce<NT>(m, true, red);
-    float ls = 0.f;
-    for (int t = threadIdx.x; t < k; t += NT) {
-      const float2 ml = s.part_ml[(int64_t)(base + t) * kDcRows + r];
-      const float wt = M == -INFINITY ? 0.f : ex2(ml.x - M);  // 0 for a piece that saw no visible key
-      w[(r - r_lo) * k + t] = wt;
-      ls += wt * ml.y;
-    }
-    const float L = dc_block_reduce<NT>(ls, false, red);
-    if (threadIdx.x == 0) {
-      Mr[r - r_lo] = M;
-      Lr[r - r_lo] = L;
-    }
+  // (m, l) of every (piece t, row r) at [t * rows + r], in one parallel
+  // pass; then one thread per row turns the maxima into the weights
+  // w = 2^(m - M) (in place) and the sum L.
+  for (int e = threadIdx.x; e < rows * k; e += NT) {
+    const float2 ml = s.part_ml[(int64_t)(base + e / rows) * kDcRows + e % rows];
+    w[e] = ml.x;
+    wl[e] = ml.y;
   }
   __syncthreads();
-  for (int it = lo + threadIdx.x; it < hi; it += NT) {
-    const int r = it / C4, c4 = it % C4;
-    const float *wr = w + (r - r_lo) * k;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
+  for (int r = threadIdx.x; r < rows; r += NT) {
+    float m = -INFINITY;
+    for (int t = 0; t < k; ++t) m = fmaxf(m, w[t * rows + r]);
+    float ls = 0.f;
     for (int t = 0; t < k; ++t) {
-      const float wt = wr[t];
-      const float4 a = reinterpret_cast<const float4 *>(s.part_acc + ((int64_t)(base + t) * kDcRows + r) * DV)[c4];
-      acc.x = fmaf(wt, a.x, acc.x);
-      acc.y = fmaf(wt, a.y, acc.y);
-      acc.z = fmaf(wt, a.z, acc.z);
-      acc.w = fmaf(wt, a.w, acc.w);
+      const float wt = m == -INFINITY ? 0.f : ex2(w[t * rows + r] - m);  // 0 for a piece that saw no visible key
+      w[t * rows + r] = wt;
+      ls += wt * wl[t * rows + r];
     }
-    const float L = Lr[r - r_lo], inv = L > 0.f ? 1.f / L : 0.f;
-    const int tok = qr.x + r / G, h = gh * G + r % G;
-    T *orow = reinterpret_cast<T *>(p.o) + (int64_t)tok * p.o_rs + (int64_t)h * p.o_hs + 4 * c4;
-    orow[0] = from_f32<T>(acc.x * inv);
-    orow[1] = from_f32<T>(acc.y * inv);
-    orow[2] = from_f32<T>(acc.z * inv);
-    orow[3] = from_f32<T>(acc.w * inv);
-    if (c4 == 0 && p.lse)
-      p.lse[(int64_t)tok * p.hq + h] = L > 0.f ? (Mr[r - r_lo] + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
+    Mr[r] = m;
+    Lr[r] = ls;
+  }
+  __syncthreads();
+  // This thread's items lo + threadIdx.x + q*NT, two at a time; the partial
+  // loads of up to eight pieces of both are issued before any is used, so
+  // up to sixteen are in flight.
+  const int nq = hi - lo > (int)threadIdx.x ? (hi - lo - 1 - (int)threadIdx.x) / NT + 1 : 0;
+  for (int q0 = 0; q0 < nq; q0 += 2) {
+    const bool two = q0 + 1 < nq;
+    int rq[2], cq[2];
+    float4 acc[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int it = lo + threadIdx.x + (q0 + (two ? q : 0)) * NT;
+      rq[q] = it % rows;
+      cq[q] = it / rows;
+      acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int t0 = 0; t0 < k; t0 += 8) {
+      float4 a[2][8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          a[q][u] = t0 + u < k ? *dc_pacc<DV>(s, base + t0 + u, rq[q], cq[q]) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const float wt = t0 + u < k ? w[(t0 + u) * rows + rq[q]] : 0.f;
+          acc[q].x = fmaf(wt, a[q][u].x, acc[q].x);
+          acc[q].y = fmaf(wt, a[q][u].y, acc[q].y);
+          acc[q].z = fmaf(wt, a[q][u].z, acc[q].z);
+          acc[q].w = fmaf(wt, a[q][u].w, acc[q].w);
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (q == 1 && !two) break;
+      const int r = rq[q], c4 = cq[q];
+      const float L = Lr[r], inv = L > 0.f ? 1.f / L : 0.f;
+      const int tok = qr.x + r / G, h = gh * G + r % G;
+      T *orow = reinterpret_cast<T *>(p.o) + (int64_t)tok * p.o_rs + (int64_t)h * p.o_hs + 4 * c4;
+      dc_store4<T>(orow, acc[q].x * inv, acc[q].y * inv, acc[q].z * inv, acc[q].w * inv);
+      if (c4 == 0 && p.lse)
+        p.lse[(int64_t)tok * p.hq + h] = L > 0.f ? (Mr[r] + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
+    }
   }
 }
 
@@ -761,10 +794,9 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
           for (int e = 0; e < 4; ++e)
             reinterpret_cast<uint4 *>(orow)[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         } else {
-          float4 *dst = reinterpret_cast<float4 *>(s.part_acc + ((int64_t)sg * kDcRows + r) * kDcDv + col);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
+            *dc_pacc<kDcDv>(s, sg, r, col / 4 + e) = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
                                  __uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
         }
       }
@@ -798,24 +830,21 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
 }
 
 // ----------------------------------------------------------------------------
-// Merge the pieces of every sequence that was split: block (row r, sequence
-// v), DV/4 threads.  Row r of sequence v = (b, g) is query token r / G of
-// batch entry b, head g*G + r % G, with G = Hq / heads.
+// Merge the pieces of every sequence that was split.  Row r of sequence
+// v = (b, g) is query token r / G of batch entry b, head g*G + r % G, with
+// G = Hq / heads.  Grid-stride over items (sequence v, block of 16 columns);
+// thread (r, q) of the 256 takes row r and columns 4(4j + q) .. +3 of item j,
+// so the partial loads of a warp are contiguous.  An item whose sequence was
+// not split (stored directly by the decode kernel) costs one load.
+constexpr int kDcCombineThreads = 256;
 template <typename T, int DV>
-__global__ void __launch_bounds__(DV) decode_combine_kernel(const AttnParams p, const DecodeSched s, int n_seq) {
-  // Grid-stride over items (sequence v, row r); an item whose sequence was
-  // not split (stored directly by the decode kernel) costs one load.  DV
-  // threads: four groups of DV/4; group q sums the pieces i = q, q+4, ...
-  // (each thread four columns), so four times as many partial loads are in
-  // flight, and the groups' sums are added in shared memory.
-  constexpr int kC = DV / 4;  // threads per group
-  __shared__ float red_m[DV];
-  __shared__ float4 red_acc[3][kC];
-  __shared__ float red_l[3];
-  const int grp = threadIdx.x / kC, col = threadIdx.x % kC;
-  const int n_items = n_seq * kDcRows;
+__global__ void __launch_bounds__(kDcCombineThreads) decode_combine_kernel(const AttnParams p, const DecodeSched s,
+                                                                           int n_seq) {
+  constexpr int kBlocks = DV / 16;  // 16-column blocks per row
+  const int r = threadIdx.x % kDcRows, q = threadIdx.x / kDcRows;
+  const int n_items = n_seq * kBlocks;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int v = item / kDcRows, r = item % kDcRows;
+    const int v = item / kBlocks, c4 = (item % kBlocks) * 4 + q;
     const int cnt = s.seg_cnt[v];
     // not split: stored directly by the decode kernel (a sequence with no
     // piece, cnt = 0, is written here: O = 0, LSE = -inf)
@@ -823,59 +852,30 @@ __global__ void __launch_bounds__(DV) decode_combine_kernel(const AttnParams p, 
     const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
     const int2 qr = dc_q(p, b);
     if (r >= qr.y * G) continue;
-    const int tok = qr.x + r / G, h = gh * G + r % G;
-    T *orow = reinterpret_cast<T *>(p.o) + (int64_t)tok * p.o_rs + (int64_t)h * p.o_hs;
     const int base = s.seg_base[v];
-    // M = the largest piece maximum (all threads take part)
-    float m = -INFINITY;
-    for (int i = threadIdx.x; i < cnt; i += DV) m = fmaxf(m, s.part_ml[(int64_t)(base + i) * kDcRows + r].x);
-    red_m[threadIdx.x] = m;
-    __syncthreads();
-    for (int w = DV / 2; w > 0; w >>= 1) {
-      if (threadIdx.x < w) red_m[threadIdx.x] = fmaxf(red_m[threadIdx.x], red_m[threadIdx.x + w]);
-      __syncthreads();
-    }
-    const float M = red_m[0];
+    float M = -INFINITY;
+    for (int i = 0; i < cnt; ++i) M = fmaxf(M, s.part_ml[(int64_t)(base + i) * kDcRows + r].x);
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (M != -INFINITY) {
 #pragma unroll 4
-      for (int i = grp; i < cnt; i += 4) {
+      for (int i = 0; i < cnt; ++i) {
         const float2 ml = s.part_ml[(int64_t)(base + i) * kDcRows + r];
         const float w = ex2(ml.x - M);  // 0 for a piece that saw no visible key
         L += w * ml.y;
-        const float4 a = reinterpret_cast<const float4 *>(s.part_acc + ((int64_t)(base + i) * kDcRows + r) * DV)[col];
+        const float4 a = *dc_pacc<DV>(s, base + i, r, c4);
         acc.x = fmaf(w, a.x, acc.x);
         acc.y = fmaf(w, a.y, acc.y);
         acc.z = fmaf(w, a.z, acc.z);
         acc.w = fmaf(w, a.w, acc.w);
       }
     }
-    if (grp > 0) {
-      red_acc[grp - 1][col] = acc;
-      if (col == 0) red_l[grp - 1] = L;
-    }
-    __syncthreads();
-    if (grp == 0) {
-#pragma unroll
-      for (int q = 0; q < 3; ++q) {
-        const float4 o = red_acc[q][col];
-        acc.x += o.x;
-        acc.y += o.y;
-        acc.z += o.z;
-        acc.w += o.w;
-        L += red_l[q];
-      }
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      const int d = col * 4;
-      orow[d + 0] = from_f32<T>(acc.x * inv);
-      orow[d + 1] = from_f32<T>(acc.y * inv);
-      orow[d + 2] = from_f32<T>(acc.z * inv);
-      orow[d + 3] = from_f32<T>(acc.w * inv);
-      if (col == 0 && p.lse)
-        p.lse[(int64_t)tok * p.hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
-    }
-    __syncthreads();  // red_m / red_acc are reused by the next item
+    const int tok = qr.x + r / G, h = gh * G + r % G;
+    T *orow = reinterpret_cast<T *>(p.o) + (int64_t)tok * p.o_rs + (int64_t)h * p.o_hs + 4 * c4;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    dc_store4<T>(orow, acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (c4 == 0 && p.lse)
+      p.lse[(int64_t)tok * p.hq + h] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994530942f : -INFINITY;
   }
 }
 

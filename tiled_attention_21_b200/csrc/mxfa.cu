@@ -370,10 +370,10 @@ DecodeSched decode_sched(const AttnParams &p, int heads, int num_splits, int dv,
 
 // `kv_rows`: rows of the K / V tensors; `box`: TMA box height (128, or the
 // page size of a paged cache with pages shorter than a tile).
-// Blocks of the combine kernel: it walks (sequence, row) items with a grid
-// stride, two blocks per SM of the decode grid at most.
-int combine_grid(int n_seq, int decode_grid) {
-  const int64_t items = (int64_t)n_seq * kDcRows;
+// Blocks of the combine kernel: it walks (sequence, 16-column block) items
+// with a grid stride, two blocks per SM of the decode grid at most.
+int combine_grid(int n_seq, int dv, int decode_grid) {
+  const int64_t items = (int64_t)n_seq * (dv / 16);
   return (int)std::max<int64_t>(1, std::min<int64_t>(items, 2 * (int64_t)decode_grid));
 }
 
@@ -403,7 +403,7 @@ mxfa_status_t launch_decode_gqa_t(AttnParams &p, const DecodeSched &s, mxfa_dtyp
   k<<<s.grid, kGqThreads, GqaCfg<D>::kSmemBytes, st>>>(p, s, mk, mv);
   MXFA_CUDA(cudaGetLastError());
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  decode_combine_kernel<T, D><<<combine_grid(n_seq, s.grid), D, 0, st>>>(p, s, n_seq);
+  decode_combine_kernel<T, D><<<combine_grid(n_seq, D, s.grid), kDcCombineThreads, 0, st>>>(p, s, n_seq);
   MXFA_CUDA(cudaGetLastError());
   return MXFA_OK;
 }
@@ -447,12 +447,12 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
     MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(attn_decode_tc_kernel<true>), kDcSmemBytes));
     attn_decode_tc_kernel<true><<<s.grid, kDcThreads, kDcSmemBytes, st>>>(p, s, mq, mkv);
     MXFA_CUDA(cudaGetLastError());
-    decode_combine_kernel<__nv_bfloat16, kDcDv><<<combine_grid(p.batch, s.grid), kDcDv, 0, st>>>(p, s, p.batch);
+    decode_combine_kernel<__nv_bfloat16, kDcDv><<<combine_grid(p.batch, kDcDv, s.grid), kDcCombineThreads, 0, st>>>(p, s, p.batch);
   } else {
     MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(attn_decode_tc_kernel<false>), kDcSmemBytes));
     attn_decode_tc_kernel<false><<<s.grid, kDcThreads, kDcSmemBytes, st>>>(p, s, mq, mkv);
     MXFA_CUDA(cudaGetLastError());
-    decode_combine_kernel<__half, kDcDv><<<combine_grid(p.batch, s.grid), kDcDv, 0, st>>>(p, s, p.batch);
+    decode_combine_kernel<__half, kDcDv><<<combine_grid(p.batch, kDcDv, s.grid), kDcCombineThreads, 0, st>>>(p, s, p.batch);
   }
   MXFA_CUDA(cudaGetLastError());
   return MXFA_OK;
