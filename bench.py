@@ -58,7 +58,10 @@ def decode_bytes(p):
     """Algorithmic bytes of one decode: the KV cache once (MLA: the shared
     latent rows; grouped-query: K and V), q, O and LSE."""
     es = 2
-    kv = p.kv.numel() * es if p.mla else (p.k.numel() + p.v.numel()) * es
+    if p.kv_scale is not None:  # E4M3 latent cache: one byte per element
+        kv = p.kv.numel()
+    else:
+        kv = p.kv.numel() * es if p.mla else (p.k.numel() + p.v.numel()) * es
     return kv + p.q.numel() * es + p.total_q * p.hq * p.dv * es + p.total_q * p.hq * 4
 
 
@@ -249,7 +252,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=128,
                     help="sequences of the MLA decode workload (128 = the full workload; smaller for captures)")
-    ap.add_argument("--only", choices=["prefill", "decode", "gqa"], default=None,
+    ap.add_argument("--only", choices=["prefill", "decode", "gqa", "fp8"], default=None,
                     help="time one workload only (used for profiling captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -288,7 +291,7 @@ def main():
         mx.mxfa_attn_fwd(q, k, v, causal=True, out=o, lse=lse, ws=ws, stream=stream)
 
     flops = prefill_flops(B, H, S, D)
-    if args.only in ("decode", "gqa"):
+    if args.only in ("decode", "gqa", "fp8"):
         args.steps = 0
     with ClockSampler(local) as clk:
         times = time_steps(step, args.steps, args.warmup, flush, stream, world)
@@ -380,6 +383,36 @@ def main():
                                    "traffic": recorded_traffic("decode_gqa", pg.name),
                                    "peak_kind": f"{pk_kind} HBM copy"}}
 
+    # ---------------- MLA decode over an E4M3 cache (next scope row; secondary measurement)
+    decode_fp8 = None
+    if not args.no_decode and args.only in (None, "fp8"):
+        pf = workloads.cfg_mla_decode_fp8()
+        df = to_dev(pf, dev)
+        of = torch.empty((pf.total_q, pf.hq, pf.dv), dtype=torch.bfloat16, device=dev)
+        lf = torch.empty((pf.total_q, pf.hq), dtype=torch.float32, device=dev)
+        need = mx.load().mxfa_attn_decode_mla_fp8kv_workspace_size(pf.batch, 4, pf.hq, 8192, 0)
+        wsf = torch.zeros(need + 256, dtype=torch.uint8, device=dev)
+
+        def fstep():
+            mx.mxfa_attn_decode_mla_fp8kv(df["q"], df["kv"], pf.kv_scale, df["cu_q"], df["cu_k"], 4, 8192,
+                                          softmax_scale=pf.scale, out=of, lse=lf, ws=wsf, stream=stream)
+
+        ftimes = time_steps(fstep, max(5, args.steps // 3), 3, lambda: None, stream, world)  # 604 MB codes >> L2
+        fbytes = decode_bytes(pf)
+        fms = max_over_ranks(statistics.mean(ftimes), world)
+        fgbs = fbytes / (fms / 1e3) / 1e9
+        fflops = 2.0 * pf.total_q * pf.hq * (pf.total_k // pf.batch) * (pf.dqk + pf.dv)
+        decode_fp8 = {"workload": pf.name, "value": fgbs * world, "unit": "GB/s", "ms_per_step": fms,
+                      "algorithmic_bytes": fbytes, "l2": "inputs (604 MB of codes) larger than L2",
+                      "kv_rows_per_s": pf.total_k * world / (fms / 1e3),
+                      "mma_tflops": fflops / (fms / 1e3) / 1e12,
+                      "roofline": {"bound": "hbm", "achieved": fgbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                   "frac": fgbs / pk["hbm_gbs"],
+                                   "traffic": recorded_traffic("decode", pf.name),
+                                   "peak_kind": f"{pk_kind} HBM copy"}}
+        if decode is not None:
+            decode["kv_rows_per_s"] = pdc.total_k * world / (decode["ms_per_step"] / 1e3)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only is None:
         cpu = cpu_baseline_prefill()
@@ -395,7 +428,7 @@ def main():
                 "e2e": None if args.only else {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                                                "d2h_bytes_per_step": d2h},
                 "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
-                "decode_gqa": decode_gqa}
+                "decode_gqa": decode_gqa, "decode_fp8": decode_fp8}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

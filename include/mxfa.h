@@ -183,6 +183,37 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
                                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * MLA split-KV decode over an fp8 latent cache (kernelbot-amd-mixed-mla
+ * submission 588924 names an fp8 KV cache in its docstring; its code reads
+ * the bf16 cache).  The page gives no fp8 format or scaling; this entry
+ * point reads it as
+ *   kv: [total_kv, 576] bytes, OCP 8-bit floating point E4M3 codes (sign,
+ *       4 exponent bits with bias 7, 3 mantissa bits, subnormals, no
+ *       infinities; the format torch calls float8_e4m3fn), row t at
+ *       kv + t*kv_row_stride (bytes, a multiple of 16, >= 576);
+ *   kv_scale: one per-tensor dequantisation factor, finite:
+ *       key / value element = kv_scale * E4M3 value of its code.
+ * The value of row t is its first 512 dequantised columns, as in
+ * mxfa_attn_decode_splitkv's MLA shape.  The codes 0x7f and 0xff (NaN) are
+ * not valid cache entries: they are read as +-480.
+ *   q: [total_q, Hq, 576] bf16 contiguous; o: [total_q, Hq, 512] bf16;
+ *   lse: [total_q, Hq] fp32 (or NULL); qo_indptr / kv_indptr, max lengths,
+ *   causal, num_splits and the workspace as for mxfa_attn_decode_splitkv.
+ *   Requires max_q_len * Hq <= 64 (else MXFA_ERR_UNSUPPORTED).  kv must be
+ *   a valid 16-byte aligned pointer even when total_kv = 0.
+ * The kernel widens each staged tile of codes to bf16 exactly in shared
+ * memory and applies kv_scale to the scores and to the outputs, so the
+ * result equals attention over the dequantised cache up to the bf16 path's
+ * rounding.
+ */
+size_t mxfa_attn_decode_mla_fp8kv_workspace_size(int batch, int max_q_len, int Hq, int max_kv_len, int num_splits);
+mxfa_status_t mxfa_attn_decode_mla_fp8kv(const void *q, const void *kv, float kv_scale, void *o, float *lse,
+                                         const int32_t *qo_indptr, const int32_t *kv_indptr, int batch, int total_q,
+                                         int total_kv, int max_q_len, int max_kv_len, int Hq, int64_t kv_row_stride,
+                                         float softmax_scale, int causal, int num_splits, void *workspace,
+                                         size_t workspace_bytes, void *stream);
+
+/*
  * Decode over a KV cache, with an optional append (mxflashattn 1.4.0 api.py,
  * flash_attn_with_kvcache: q, k_cache, v_cache, k, v, cache_seqlens,
  * block_table, causal).

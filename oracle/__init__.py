@@ -109,6 +109,15 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_q, cu_k, sca
 
 
 def problem(p, pairs=None, threads=None, lib=None, return_psum=False):
-    """Run the oracle on a ``workloads.Problem`` (inputs in their stored dtype)."""
+    """Run the oracle on a ``workloads.Problem`` (inputs in their stored dtype).
+    An E4M3 latent cache (``p.kv_scale`` set, ``p.kv`` the codes) is first
+    dequantised exactly in fp64 (``e4m3.dequantize``); q is then taken in fp64
+    too (exact), since the oracle wants one dtype for q, k and v."""
+    if getattr(p, "kv_scale", None) is not None:
+        from . import e4m3
+        kv = e4m3.dequantize(p.kv, p.kv_scale)
+        tk = kv.shape[0]
+        return attention(p.q.double(), kv.view(tk, 1, p.dqk), kv[:, :p.dv].view(tk, 1, p.dv), p.cu_q, p.cu_k,
+                         p.scale, p.causal, pairs=pairs, threads=threads, lib=lib, return_psum=return_psum)
     return attention(p.q, p.k, p.v, p.cu_q, p.cu_k, p.scale, p.causal, pairs=pairs,
                      threads=threads, lib=lib, return_psum=return_psum)

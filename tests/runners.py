@@ -30,6 +30,10 @@ def run(p, d, entry=None, num_splits=0, stream=None, out=None, lse=None):
         return mx.mxfa_attn_varlen_fwd(d["q"], d["k"], d["v"], d["cu_q"], d["cu_k"], max(p.seqlens_q()),
                                        max(p.seqlens_k()), causal=p.causal, softmax_scale=p.scale, stream=stream,
                                        out=out, lse=lse)
+    if p.kv_scale is not None:
+        return mx.mxfa_attn_decode_mla_fp8kv(d["q"], d["kv"], p.kv_scale, d["cu_q"], d["cu_k"], max(p.seqlens_q()),
+                                             max(p.seqlens_k()), softmax_scale=p.scale, causal=p.causal,
+                                             num_splits=num_splits, stream=stream, out=out, lse=lse)
     return mx.mxfa_attn_decode_splitkv(d["q"], d["k"], d["v"], d["cu_q"], d["cu_k"], max(p.seqlens_q()),
                                        max(p.seqlens_k()), softmax_scale=p.scale, causal=p.causal,
                                        num_splits=num_splits, stream=stream, out=out, lse=lse)

@@ -96,6 +96,31 @@ def test_varlen_and_decode_validation(lib):
     assert r == m.MXFA_ERR_INVALID_ARG  # negative split count
 
 
+def test_fp8_decode_validation(lib):
+    import tiled_attention_21_b200 as m
+
+    def c(**kw):
+        a = dict(q=FAKE, kv=FAKE, ks=0.25, o=FAKE, lse=None, qo=FAKE, kvi=FAKE, B=2, tq=8, tkv=64, mq=4, mkv=32,
+                 Hq=16, rs=576, scale=float("nan"), causal=0, splits=0, ws=FAKE, wn=1 << 20)
+        a.update(kw)
+        return lib.mxfa_attn_decode_mla_fp8kv(a["q"], a["kv"], a["ks"], a["o"], a["lse"], a["qo"], a["kvi"], a["B"],
+                                              a["tq"], a["tkv"], a["mq"], a["mkv"], a["Hq"], a["rs"], a["scale"],
+                                              a["causal"], a["splits"], a["ws"], a["wn"], None)
+
+    assert c(Hq=32) == m.MXFA_ERR_UNSUPPORTED               # 4 x 32 query rows per sequence > 64
+    assert c(ks=float("inf")) == m.MXFA_ERR_INVALID_ARG     # scale not finite
+    assert c(ks=float("nan")) == m.MXFA_ERR_INVALID_ARG
+    assert c(rs=560) == m.MXFA_ERR_INVALID_ARG              # row shorter than 576 codes
+    assert c(rs=584) == m.MXFA_ERR_INVALID_ARG              # not a multiple of 16 bytes
+    assert c(kv=None) == m.MXFA_ERR_INVALID_ARG
+    assert c(kvi=None) == m.MXFA_ERR_INVALID_ARG
+    assert c(splits=-1) == m.MXFA_ERR_INVALID_ARG
+    assert c(wn=16) == m.MXFA_ERR_WORKSPACE
+    assert c(B=0) == m.MXFA_OK                              # nothing to do
+    need = lib.mxfa_attn_decode_mla_fp8kv_workspace_size(128, 4, 16, 8192, 0)
+    assert need > 256 and need == lib.mxfa_attn_decode_splitkv_workspace_size(128, 4, 16, 1, 512, 8192, 0, 2)
+
+
 def test_workspace_sizes(lib):
     assert lib.mxfa_attn_fwd_workspace_size(4, 2048, 2048, 16, 16, 128, 2) >= 256
     small = lib.mxfa_attn_varlen_fwd_workspace_size(2, 128, 128, 8, 128, 2)

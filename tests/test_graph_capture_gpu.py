@@ -75,3 +75,10 @@ def test_graph_varlen_prefill():
     a = workloads.varlen(57, lens, lens, 8, 2, 128, "bf16", True)
     b = workloads.varlen(58, lens, lens, 8, 2, 128, "bf16", True)
     _replay_matches(a, b, "varlen")
+
+
+def test_graph_mla_decode_fp8kv():
+    a = workloads.mla_decode_fp8(59, batch=4, q_len=4, kv_len=1024)
+    b = workloads.mla_decode_fp8(60, batch=4, q_len=4, kv_len=1024)
+    b.kv_scale = a.kv_scale  # the scale is a call argument, captured with the graph
+    _replay_matches(a, b, "decode")

@@ -312,3 +312,64 @@ def test_pins_catch_planted_mistake(mutant, tmp_path):
         except (AssertionError, RuntimeError):
             caught.append(pin.__name__)
     assert caught, f"mutant {mutant} ({MUTANTS[mutant]}) passed every pin"
+
+
+# ---------------------------------------------------------------------------
+# E4M3 codes (oracle/e4m3.py) and the oracle over an fp8 latent cache
+# ---------------------------------------------------------------------------
+
+def test_e4m3_closed_forms():
+    """Values the E4M3 definition fixes by itself."""
+    from oracle import e4m3
+    assert e4m3.value(0x00) == 0.0 and math.copysign(1.0, e4m3.value(0x00)) == 1.0
+    assert e4m3.value(0x80) == 0.0 and math.copysign(1.0, e4m3.value(0x80)) == -1.0
+    assert e4m3.value(0x38) == 1.0           # exponent field = bias, mantissa 0
+    assert e4m3.value(0xB8) == -1.0
+    assert e4m3.value(0x3C) == 1.5
+    assert e4m3.value(0x7E) == 448.0         # largest finite value
+    assert e4m3.value(0x08) == 2.0 ** -6     # smallest normal
+    assert e4m3.value(0x01) == 2.0 ** -9     # smallest subnormal
+    assert e4m3.value(0x07) == 7 * 2.0 ** -9  # largest subnormal
+    assert math.isnan(e4m3.value(0x7F)) and math.isnan(e4m3.value(0xFF))
+
+
+def test_e4m3_matches_torch_float8_for_every_code():
+    """torch's own float8_e4m3fn -> float64 conversion, written independently
+    of oracle/e4m3.py, agrees on all 256 codes (signs of zero included)."""
+    from oracle import e4m3
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64)
+    got = e4m3.decode(codes)
+    nan = torch.isnan(ref)
+    assert torch.equal(nan, torch.isnan(got)) and int(nan.sum()) == 2
+    assert torch.equal(got[~nan], ref[~nan])
+    assert torch.equal(torch.signbit(got[~nan]), torch.signbit(ref[~nan]))
+
+
+def test_e4m3_order_and_sign():
+    from oracle import e4m3
+    vals = [e4m3.value(c) for c in range(0x7F)]
+    assert all(a < b for a, b in zip(vals, vals[1:]))
+    assert all(e4m3.value(c | 0x80) == -e4m3.value(c) for c in range(0x7F))
+
+
+def test_fp8_mla_oracle_matches_brute_force():
+    """oracle.problem over an E4M3 cache equals the pure-Python restatement
+    given torch's own dequantisation (torch's float8 cast times the scale,
+    value = the first 512 columns)."""
+    p = workloads.mla_decode_fp8(31, batch=2, q_len=2, kv_len=0, heads=2, lens_kv=[3, 5], causal=True)
+    o, lse = oracle.problem(p)
+    kv = p.kv.view(torch.float8_e4m3fn).to(torch.float64) * p.kv_scale
+    bo, bl = brute.attention_packed(p.q.double().tolist(), kv.view(-1, 1, 576).tolist(),
+                                    kv[:, :512].reshape(-1, 1, 512).tolist(), p.cu_q.tolist(), p.cu_k.tolist(),
+                                    p.scale, p.causal)
+    assert torch.allclose(o, torch.tensor(bo, dtype=torch.float64), rtol=0, atol=1e-12)
+    assert torch.allclose(lse, torch.tensor(bl, dtype=torch.float64), rtol=0, atol=1e-12)
+
+
+def test_fp8_workload_codes_are_finite_and_span_the_range():
+    p = workloads.mla_decode_fp8(32, batch=2, q_len=4, kv_len=300)
+    vals = p.kv.view(torch.float8_e4m3fn).to(torch.float64)
+    assert not torch.isnan(vals).any()
+    assert vals.abs().max().item() == 448.0
+    assert p.kv.dtype == torch.uint8 and tuple(p.kv.shape) == (600, 576)

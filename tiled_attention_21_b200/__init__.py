@@ -9,6 +9,7 @@ Functions carry the C entry points' names:
     mxfa_attn_fwd(q, k, v, causal=..., softmax_scale=...)              -> (o, lse)
     mxfa_attn_varlen_fwd(q, k, v, cu_q, cu_k, max_q, max_k, ...)       -> (o, lse)
     mxfa_attn_decode_splitkv(q, k, v, qo_indptr, kv_indptr, ...)       -> (o, lse)
+    mxfa_attn_decode_mla_fp8kv(q, kv, kv_scale, qo_indptr, kv_indptr, ...) -> (o, lse)
 """
 from __future__ import annotations
 
@@ -56,6 +57,11 @@ def load():
             lib.mxfa_attn_decode_splitkv.restype = i32
             lib.mxfa_attn_decode_splitkv_workspace_size.argtypes = [i32] * 8
             lib.mxfa_attn_decode_splitkv_workspace_size.restype = sz
+            lib.mxfa_attn_decode_mla_fp8kv.argtypes = [vp, vp, f32] + [vp] * 4 + [i32] * 6 + [i64, f32, i32, i32,
+                                                                                        vp, sz, vp]
+            lib.mxfa_attn_decode_mla_fp8kv.restype = i32
+            lib.mxfa_attn_decode_mla_fp8kv_workspace_size.argtypes = [i32] * 5
+            lib.mxfa_attn_decode_mla_fp8kv_workspace_size.restype = sz
             lib.mxfa_attn_decode_kvcache.argtypes = [vp] * 7 + [i32] * 10 + [i32, f32, i32, i32, vp, vp, vp, sz, vp]
             lib.mxfa_attn_decode_kvcache.restype = i32
             lib.mxfa_attn_decode_kvcache_workspace_size.argtypes = [i32] * 8
@@ -204,6 +210,37 @@ def mxfa_attn_decode_splitkv(q, k, v, qo_indptr, kv_indptr, max_q_len: int, max_
                                         _ptr(kv_indptr), batch, total_q, total_kv, int(max_q_len), int(max_kv_len),
                                         Hq, Hkv, Dqk, Dv, k.stride(0), v.stride(0), dt, _scale(softmax_scale),
                                         int(bool(causal)), int(num_splits), wp, wn, _stream(stream)))
+    return out, lse
+
+
+def mxfa_attn_decode_mla_fp8kv(q, kv, kv_scale: float, qo_indptr, kv_indptr, max_q_len: int, max_kv_len: int,
+                               softmax_scale: float | None = None, causal: bool = False, num_splits: int = 0,
+                               out=None, lse=None, return_lse: bool = True, ws: torch.Tensor | None = None,
+                               stream=None):
+    """MLA decode over an E4M3 latent cache.  q [total_q, Hq, 576] bf16 contiguous;
+    kv [total_kv, 576] torch.float8_e4m3fn or uint8 codes (unit stride inside a
+    row); element value = kv_scale * code value.  Returns (o [total_q, Hq, 512]
+    bf16, lse [total_q, Hq])."""
+    lib = load()
+    total_q, Hq, Dqk = q.shape
+    total_kv = kv.shape[0]
+    if q.dtype != torch.bfloat16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16")
+    if kv.dtype not in (torch.uint8, torch.float8_e4m3fn) or kv.dim() != 2 or kv.stride(1) != 1:
+        raise ValueError("kv must be [total_kv, 576] E4M3 codes with unit stride inside a row")
+    batch = qo_indptr.numel() - 1
+    if out is None:
+        out = torch.empty((total_q, Hq, 512), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((total_q, Hq), dtype=torch.float32, device=q.device)
+    need = lib.mxfa_attn_decode_mla_fp8kv_workspace_size(batch, max_q_len, Hq, max_kv_len, num_splits)
+    ws = ws if ws is not None else workspace(need, q.device)
+    wp, wn = _ws_view(ws)
+    _check(lib.mxfa_attn_decode_mla_fp8kv(_ptr(q), _ptr(kv), float(kv_scale), _ptr(out), _ptr(lse),
+                                          _ptr(qo_indptr), _ptr(kv_indptr), batch, total_q, total_kv,
+                                          int(max_q_len), int(max_kv_len), Hq, kv.stride(0),
+                                          _scale(softmax_scale), int(bool(causal)), int(num_splits), wp, wn,
+                                          _stream(stream)))
     return out, lse
 
 

@@ -89,6 +89,10 @@ struct DecodeSched {
   // counts the pieces that have stored theirs (zeroed before the launch).
   int arith_k;
   int *sync;
+  // Factor of every stored output and partial accumulator: 1, or the KV
+  // dequantisation scale of the fp8-KV MLA kernel (the scores' share of that
+  // scale is folded into AttnParams::scale_log2 by the host).
+  float o_scale;
 };
 
 // Queries of batch entry b: (first row, count); packed (cu_q) or uniform.
@@ -115,6 +119,8 @@ __device__ __forceinline__ int dc_krow(const AttnParams &p, const DecodeSched &s
 struct DecodeCtrl {
   uint64_t q_ready;
   uint64_t tile_full[kDcRingTiles], tile_empty[kDcRingTiles];
+  uint64_t stage_full[kDcRingTiles];  // fp8 KV: the slot's codes have landed
+  uint64_t low_full[kDcRingTiles];    // fp8 KV: bf16 chunks 0-3 of the slot are written
   uint64_t s_full, s_free, p_full, o_done, o_empty;
   uint64_t drain;
   uint32_t tmem_base;
@@ -123,7 +129,7 @@ struct DecodeCtrl {
 
 enum : uint32_t {
   kDSiteSlotEmpty = 0x301, kDSiteQReady, kDSiteSlotFull, kDSitePFull, kDSiteOEmpty, kDSiteSFull,
-  kDSiteODone, kDSiteSFree, kDSiteMerge
+  kDSiteODone, kDSiteSFree, kDSiteMerge, kDSiteStageFull
 };
 
 __device__ __forceinline__ int dc_range_start(int c, int T, int G) { return (int)(((int64_t)c * T) / G); }
@@ -452,14 +458,54 @@ __device__ void dc_zero_rows(const AttnParams &p, const DecodeSched &s, int v) {
 }
 
 // ----------------------------------------------------------------------------
-template <bool BF16>
-__global__ void __launch_bounds__(kDcThreads, 1)
+// ----------------------------------------------------------------------------
+// fp8 KV (OCP 8-bit floating point, E4M3: sign, 4 exponent bits with bias 7,
+// 3 mantissa bits, subnormals, no infinities).  A tile's codes (nine
+// unswizzled 64 keys x 64-byte column chunks, 36,864 bytes) land by TMA in
+// the upper half of the ring slot that will hold the tile in bf16; a
+// widening warpgroup turns them in place into the nine 64 x 128-byte,
+// 128B-swizzled bf16 chunks the MMA reads.  The bf16 chunks 0-3 end below
+// the codes; chunks 4-8 overwrite codes, so those are read into registers
+// before any of them is written.
+constexpr int kDcStageChunkBytes = kDcKeys * 64;
+constexpr int kDcStageBytes = kDcChunks * kDcStageChunkBytes;  // 36,864
+constexpr int kDcStageOff = kDcChunks * kDcChunkBytes - kDcStageBytes;  // codes: upper half of the slot
+static_assert(4 * kDcChunkBytes <= kDcStageOff, "bf16 chunks 0-3 end below the staged codes");
+constexpr int kDcThreadsFp8 = 384;  // + warps 8-11: the widening warpgroup
+
+// Four E4M3 codes (the bytes of w, lowest first) to four bf16 values, exactly.
+// Code byte c becomes the 16-bit pattern sign(c) << 15 | (c & 0x7f) << 4: the
+// E4M3 exponent and mantissa fields become the low four bits of bf16's
+// exponent and the top three of its mantissa, i.e. the bf16 value is the E4M3
+// value times 2^-120 (E4M3 subnormals become bf16 subnormals), and one bf16x2
+// multiply by 2^120 restores it.  prmt builds (c, sign-fill(c)) byte pairs,
+// so the shift puts the sign in bit 15; the mask clears the rest.  The two
+// NaN codes (0x7f, 0xff) come out as +-480.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  uint32_t a, b;
+  asm("prmt.b32 %0, %1, 0, 0x9180;" : "=r"(a) : "r"(w));
+  asm("prmt.b32 %0, %1, 0, 0xB3A2;" : "=r"(b) : "r"(w));
+  a = (a << 4) & 0x87F087F0u;
+  b = (b << 4) & 0x87F087F0u;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(0x7B807B80u));  // 0x7B80 = 2^120
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(0x7B807B80u));
+}
+
+// FP8 = true: the KV cache holds E4M3 codes (tm_kv is a byte map, box 64 x 64,
+// no swizzle), staged in the ring slots and widened there by warps 8-11 (384
+// threads); from there the MMA and softmax roles run unchanged.  The
+// dequantisation scale multiplies the scores (through p.scale_log2) and the
+// outputs (s.o_scale).
+template <bool BF16, bool FP8 = false>
+__global__ void __launch_bounds__(FP8 ? kDcThreadsFp8 : kDcThreads, 1)
 attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
                       const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv) {
+  static_assert(!FP8 || BF16, "fp8 KV is widened to bf16");
+  constexpr int RT = kDcRingTiles;
   extern __shared__ uint8_t smem_raw[];
   DecodeCtrl *ctrl = reinterpret_cast<DecodeCtrl *>(smem_raw);
   const uint32_t tiles_u32 = (smem_u32(smem_raw) + 1024u + 1023u) & ~1023u;
-  const uint32_t ring_u32 = tiles_u32;                               // 3 tiles x 9 KV chunks
+  const uint32_t ring_u32 = tiles_u32;                               // RT tiles x 9 KV chunks
   const uint32_t p_u32 = ring_u32 + kDcSlots * kDcChunkBytes;        // P: 64 rows x 128 B
   uint8_t *p_gen = smem_raw + (p_u32 - smem_u32(smem_raw));
 
@@ -468,14 +514,18 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
   WsHeader *hdr = p.hdr;
   auto b_tf = [&](int x) { return smem_u32(&ctrl->tile_full[x]); };
   auto b_te = [&](int x) { return smem_u32(&ctrl->tile_empty[x]); };
+  auto b_gf = [&](int x) { return smem_u32(&ctrl->stage_full[x]); };
+  auto b_lf = [&](int x) { return smem_u32(&ctrl->low_full[x]); };
   const uint32_t b_qr = smem_u32(&ctrl->q_ready), b_sf = smem_u32(&ctrl->s_full), b_sx = smem_u32(&ctrl->s_free);
   const uint32_t b_pf = smem_u32(&ctrl->p_full), b_od = smem_u32(&ctrl->o_done), b_oe = smem_u32(&ctrl->o_empty);
 
   if (threadIdx.x == 0) {
     mbar_init(b_qr, 128);
-    for (int x = 0; x < kDcRingTiles; ++x) {
-      mbar_init(b_tf(x), 1);
+    for (int x = 0; x < RT; ++x) {
+      mbar_init(b_tf(x), FP8 ? 128 : 1);  // fp8: the 128 widening threads arrive
       mbar_init(b_te(x), 1);
+      mbar_init(b_gf(x), 1);
+      mbar_init(b_lf(x), 128);
     }
     mbar_init(b_sf, 1);
     mbar_init(b_sx, 128);
@@ -525,22 +575,34 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
                                (uint32_t)(rn * kDcDqk * 2));
         }
         for (int j = sd.y; ok && j < sd.z; ++j, ++tc) {
-          const int x = tc % kDcRingTiles;
-          if (!wait_bar(b_te(x), ((tc / kDcRingTiles) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty)) {
+          const int x = tc % RT;
+          if (!wait_bar(b_te(x), ((tc / RT) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(b_tf(x), kDcChunks * kDcChunkBytes);
-          for (int c = 0; c < kDcChunks; ++c)
-            tma_load_2d(ring_u32 + (x * kDcChunks + c) * kDcChunkBytes, &tm_kv, b_tf(x), c * 64, k0 + j * kDcKeys);
+          if (FP8) {  // the codes, into the upper half of the slot
+            mbar_arrive_expect_tx(b_gf(x), kDcStageBytes);
+            for (int c = 0; c < kDcChunks; ++c)
+              tma_load_2d(ring_u32 + x * kDcChunks * kDcChunkBytes + kDcStageOff + c * kDcStageChunkBytes, &tm_kv,
+                          b_gf(x), c * 64, k0 + j * kDcKeys);
+            // Tile j + 2 into L2, so that its load (issued once its slot is
+            // free) does not wait on HBM: the widening adds to the time from
+            // a free slot to a ready tile, which three slots must cover.
+            if (j + 2 < sd.z)
+              for (int c = 0; c < kDcChunks; ++c) tma_prefetch_2d(&tm_kv, c * 64, k0 + (j + 2) * kDcKeys);
+          } else {
+            mbar_arrive_expect_tx(b_tf(x), kDcChunks * kDcChunkBytes);
+            for (int c = 0; c < kDcChunks; ++c)
+              tma_load_2d(ring_u32 + (x * kDcChunks + c) * kDcChunkBytes, &tm_kv, b_tf(x), c * 64, k0 + j * kDcKeys);
+          }
         }
       }
       // Teardown: every tile load this thread issued must have landed.
       const uint64_t t0 = global_ns();
-      for (int x = 0; x < kDcRingTiles; ++x) {
-        const uint32_t uses = tc / kDcRingTiles + ((uint32_t)x < tc % kDcRingTiles ? 1u : 0u);
+      for (int x = 0; x < RT; ++x) {
+        const uint32_t uses = tc / RT + ((uint32_t)x < tc % RT ? 1u : 0u);
         if (uses == 0) continue;
-        while (!mbar_test(b_tf(x), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        while (!mbar_test(FP8 ? b_gf(x) : b_tf(x), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
         }
       }
     }
@@ -570,16 +632,35 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       const uint32_t p_lo0 = desc_lo(make_sdesc_sw128(p_u32, 16, 1024));
       // S of tile counter `t` into the three chains (chunk c accumulates into chain c % 3).
       auto issue_s = [&](uint32_t t) -> bool {
-        const int x = t % kDcRingTiles;
-        if (!wait_warp(b_tf(x), (t / kDcRingTiles) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
-        tc_fence_after();
+        const int x = t % RT;
         const uint32_t k_lo = k_lo0 + (uint32_t)((x * kDcChunks * kDcChunkBytes) >> 4);
+        auto mma_chunk = [&](int c, int kk) {
+          if (leader) mma_ts2(s_tmem + (c % 3) * kDcKeys, s_tmem + kDcQCol + (c * 4 + kk) * 8,
+                  k_lo + (uint32_t)((c * kDcChunkBytes + kk * 32) >> 4), k_hi, idesc_s, (c >= 3 || kk > 0) ? 1u : 0u);
+        };
+        if (FP8) {
+          // chunks 0-3 as soon as they are widened, then 4-8 (the first MMA
+          // into each chain, c = 0, 1, 2 at kk = 0, still comes first)
+          if (!wait_warp(b_lf(x), (t / RT) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
+          for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-          for (int c = 0; c < kDcChunks; ++c)
-            if (leader) mma_ts2(s_tmem + (c % 3) * kDcKeys, s_tmem + kDcQCol + (c * 4 + kk) * 8,
-                    k_lo + (uint32_t)((c * kDcChunkBytes + kk * 32) >> 4), k_hi, idesc_s, (c >= 3 || kk > 0) ? 1u : 0u);
+            for (int c = 0; c < 4; ++c) mma_chunk(c, kk);
+          if (!wait_warp(b_tf(x), (t / RT) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int c = 4; c < kDcChunks; ++c) mma_chunk(c, kk);
+        } else {
+          if (!wait_warp(b_tf(x), (t / RT) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+            for (int c = 0; c < kDcChunks; ++c) mma_chunk(c, kk);
+        }
         if (leader) mma_commit(b_sf);
         return true;
       };
@@ -607,7 +688,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
             break;
           }
           tc_fence_after();
-          const uint32_t v_lo = v_lo0 + (uint32_t)(((tc % kDcRingTiles) * kDcChunks * kDcChunkBytes) >> 4);
+          const uint32_t v_lo = v_lo0 + (uint32_t)(((tc % RT) * kDcChunks * kDcChunkBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
@@ -616,7 +697,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
                       v_lo + (uint32_t)((half * 4 * kDcChunkBytes + kk * 16 * 128) >> 4), v_hi, idesc_o,
                       (jj > 0 || kk > 0) ? 1u : 0u);
           if (leader) mma_commit(b_od);
-          if (leader) mma_commit(b_te(tc % kDcRingTiles));
+          if (leader) mma_commit(b_te(tc % RT));
         }
         ++o_uses;
       }
@@ -625,7 +706,66 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < kWaitBudgetNs) {
       }
     }
-  } else if (warp >= 4) {
+  } else if (FP8 && warp >= 8) {
+    // ------------------------------------------------------------ fp8 -> bf16 widening (warps 8-11)
+    // Per tile 2,304 groups of 16 codes g = (chunk c, key row, u) = 256c +
+    // 4 row + u: columns 16u..16u+15 of key `row` in chunk c, which become
+    // 16-byte units 2u and 2u+1 of that row of bf16 chunk c, placed by the
+    // 128B swizzle (unit ^ (row & 7)).  Thread t takes groups t + 128i:
+    // eight consecutive threads read 128 contiguous bytes and write eight
+    // distinct units of two rows, so neither side has bank conflicts.
+    const int t = threadIdx.x - 256;
+    uint8_t *ring = smem_raw + (ring_u32 - smem_u32(smem_raw));
+    auto put = [&](uint8_t *slot, int g, const uint4 &w) {
+      const int c = g >> 8, row = (g >> 2) & 63, u = g & 3;
+      uint4 a, b;
+      e4m3x4_to_bf16x4(w.x, a.x, a.y);
+      e4m3x4_to_bf16x4(w.y, a.z, a.w);
+      e4m3x4_to_bf16x4(w.z, b.x, b.y);
+      e4m3x4_to_bf16x4(w.w, b.z, b.w);
+      uint8_t *drow = slot + c * kDcChunkBytes + row * 128;
+      *reinterpret_cast<uint4 *>(drow + (((2 * u) ^ (row & 7)) << 4)) = a;
+      *reinterpret_cast<uint4 *>(drow + (((2 * u + 1) ^ (row & 7)) << 4)) = b;
+    };
+    uint32_t tc = 0;
+    bool ok = true;
+    for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
+      const int4 sd = dc_seg(p, s, sg);
+      for (int j = sd.y; j < sd.z; ++j, ++tc) {
+        const int y = tc % RT;
+        // The four warps give up together (an AND over the warpgroup), so
+        // none of them is left waiting at the named barrier below.
+        const uint32_t got = wait_bar(b_gf(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull) ? 1u : 0u;
+        uint32_t all;
+        asm volatile(
+            "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+            : "=r"(all)
+            : "r"(got)
+            : "memory");
+        if (!all) {
+          ok = false;
+          break;
+        }
+        uint8_t *slot = ring + y * kDcChunks * kDcChunkBytes;
+        const uint4 *codes = reinterpret_cast<const uint4 *>(slot + kDcStageOff);  // group g at codes[g]
+        // chunks 0-3 (groups 0-1023): their bf16 rows end below the codes
+#pragma unroll 4
+        for (int i = 0; i < 8; ++i) put(slot, t + 128 * i, codes[t + 128 * i]);
+        fence_proxy_async_smem();
+        mbar_arrive(b_lf(y));  // S may start on chunks 0-3
+        // chunks 4-8 (groups 1024-2303) overwrite codes: every thread reads
+        // its groups (and has read its chunk 0-3 groups) before any write
+        uint4 w[10];
+#pragma unroll
+        for (int i = 0; i < 10; ++i) w[i] = codes[1024 + t + 128 * i];
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+        for (int i = 0; i < 10; ++i) put(slot, 1024 + t + 128 * i, w[i]);
+        fence_proxy_async_smem();  // the MMA reads the chunks through the async proxy
+        mbar_arrive(b_tf(y));
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ softmax / epilogue
     const int sub = warp & 3, half = lane >> 4;
     const int r = sub * 16 + (lane & 15);                    // query row of this thread
@@ -776,7 +916,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       const bool direct = dc_seg_cnt(p, s, b) == 1;
       const int tok = q0 + (valid ? r / p.hq : 0), h = valid ? r % p.hq : 0;
       using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l > 0.f ? (FP8 ? s.o_scale : 1.f) / l : 0.f;
 #pragma unroll 1
       for (int q = 0; q < kDcDv / 64; ++q) {
         uint32_t ov[32];
@@ -794,6 +934,10 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
           for (int e = 0; e < 4; ++e)
             reinterpret_cast<uint4 *>(orow)[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         } else {
+          if (FP8) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * s.o_scale);
+          }
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             *dc_pacc<kDcDv>(s, sg, r, col / 4 + e) = make_float4(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]),
@@ -824,8 +968,9 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
     const int v = blockIdx.x / s.arith_k, i = blockIdx.x % s.arith_k, k = dc_seg_cnt(p, s, v);
     float *scratch = reinterpret_cast<float *>(smem_raw + kDcCtrlBytes);
-    if (k > 1 && i < k) dc_merge_pieces<T, kDcDv, kDcThreads>(p, s, v, i, k, scratch);
-    else if (k == 0 && i == 0) dc_zero_rows<T, kDcDv, kDcThreads>(p, s, v);
+    constexpr int NT = FP8 ? kDcThreadsFp8 : kDcThreads;
+    if (k > 1 && i < k) dc_merge_pieces<T, kDcDv, NT>(p, s, v, i, k, scratch);
+    else if (k == 0 && i == 0) dc_zero_rows<T, kDcDv, NT>(p, s, v);
   }
 }
 

@@ -173,6 +173,23 @@ mxfa_status_t make_map_2d(CUtensorMap *map, const void *base, mxfa_dtype_t dt, i
   return MXFA_OK;
 }
 
+// 2-D map over [rows][cols] bytes (E4M3 codes, row stride in bytes), box =
+// 64 rows x 64 bytes, no swizzle; rows past `rows` read as zero.
+mxfa_status_t make_map_2d_u8(CUtensorMap *map, const void *base, int cols, int64_t rows, int64_t row_stride) {
+  EncodeTiledFn enc;
+  mxfa_status_t st = get_encoder(&enc);
+  if (st != MXFA_OK) return st;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MXFA_ERR_INVALID_ARG, "cuTensorMapEncodeTiled (bytes) failed (%d)", (int)r);
+  return MXFA_OK;
+}
+
 // ---------------------------------------------------------------- validation
 mxfa_status_t check_ptr(const void *p, const char *name, bool allow_null = false) {
   if (!p) return allow_null ? MXFA_OK : fail(MXFA_ERR_INVALID_ARG, "%s is NULL", name);
@@ -358,6 +375,7 @@ DecodeSched decode_sched(const AttnParams &p, int heads, int num_splits, int dv,
   s.kv_len = reinterpret_cast<int *>(base + w.kv_len);
   s.sync = reinterpret_cast<int *>(base + w.sync);
   s.arith_k = 0;
+  s.o_scale = 1.f;
   s.max_segs = w.max_segs;
   s.num_splits = num_splits;
   s.grid = std::min(sms, kDcMaxGrid);
@@ -418,14 +436,26 @@ mxfa_status_t launch_decode_gqa(AttnParams &p, const DecodeSched &s, mxfa_dtype_
             : launch_decode_gqa_t<64, false>(p, s, dt, kv_rows, box, st);
 }
 
+// The MLA tensor-core decode.  kv_fp8: the cache holds E4M3 codes
+// (row stride p.k_rs bytes) with dequantisation scale o_scale, and q / o are
+// bf16; otherwise it holds `dt` values.
 mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int total_kv, int num_splits, void *ws,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool kv_fp8 = false, float o_scale = 1.f) {
   int sms = 0;
   MXFA_TRY(sm_count(&sms));
-  const DecodeSched s = decode_sched(p, 1, num_splits, kDcDv, kDcKeys, ws, sms);
+  DecodeSched s = decode_sched(p, 1, num_splits, kDcDv, kDcKeys, ws, sms);
+  s.o_scale = o_scale;
   CUtensorMap mq, mkv;
   MXFA_TRY(make_map_2d(&mq, p.q, dt, kDcDqk, (int64_t)total_q * p.hq, kDcDqk));
-  MXFA_TRY(make_map_2d(&mkv, p.k, dt, kDcDqk, total_kv, p.k_rs));
+  if (kv_fp8)
+    MXFA_TRY(make_map_2d_u8(&mkv, p.k, kDcDqk, total_kv, p.k_rs));
+  else
+    MXFA_TRY(make_map_2d(&mkv, p.k, dt, kDcDqk, total_kv, p.k_rs));
+  const void *k = kv_fp8 ? reinterpret_cast<const void *>(attn_decode_tc_kernel<true, true>)
+                  : dt == MXFA_BF16 ? reinterpret_cast<const void *>(attn_decode_tc_kernel<true>)
+                                    : reinterpret_cast<const void *>(attn_decode_tc_kernel<false>);
+  MXFA_TRY(ensure_smem(k, kDcSmemBytes));
+  const int threads = kv_fp8 ? kDcThreadsFp8 : kDcThreads;
   // Small problems run in one launch: no prep kernel (the pieces follow from
   // kv_indptr) and no combine kernel (split sequences merge in the kernel).
   const int max_tiles = (p.max_sk + kDcKeys - 1) / kDcKeys;
@@ -434,26 +464,19 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
     const int t_min = max_tiles > 32 ? 4 : 2;  // tiles per piece at least (merge cost vs chain length)
     sa.arith_k = std::max(1, std::min(s.grid / p.batch, (max_tiles + t_min - 1) / t_min));
     if (sa.arith_k > 1) MXFA_CUDA(cudaMemsetAsync(sa.sync, 0, sizeof(int) * (size_t)p.batch, st));
-    const void *k = dt == MXFA_BF16 ? reinterpret_cast<const void *>(attn_decode_tc_kernel<true>)
-                                    : reinterpret_cast<const void *>(attn_decode_tc_kernel<false>);
-    MXFA_TRY(ensure_smem(k, kDcSmemBytes));
     void *args[] = {&p, &sa, &mq, &mkv};
-    MXFA_CUDA(cudaLaunchCooperativeKernel(k, dim3(p.batch * sa.arith_k), dim3(kDcThreads), args, kDcSmemBytes, st));
+    MXFA_CUDA(cudaLaunchCooperativeKernel(k, dim3(p.batch * sa.arith_k), dim3(threads), args, kDcSmemBytes, st));
     return MXFA_OK;
   }
   decode_prep_kernel<<<1, 1024, 0, st>>>(p, s);
   MXFA_CUDA(cudaGetLastError());
-  if (dt == MXFA_BF16) {
-    MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(attn_decode_tc_kernel<true>), kDcSmemBytes));
-    attn_decode_tc_kernel<true><<<s.grid, kDcThreads, kDcSmemBytes, st>>>(p, s, mq, mkv);
-    MXFA_CUDA(cudaGetLastError());
-    decode_combine_kernel<__nv_bfloat16, kDcDv><<<combine_grid(p.batch, kDcDv, s.grid), kDcCombineThreads, 0, st>>>(p, s, p.batch);
-  } else {
-    MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(attn_decode_tc_kernel<false>), kDcSmemBytes));
-    attn_decode_tc_kernel<false><<<s.grid, kDcThreads, kDcSmemBytes, st>>>(p, s, mq, mkv);
-    MXFA_CUDA(cudaGetLastError());
-    decode_combine_kernel<__half, kDcDv><<<combine_grid(p.batch, kDcDv, s.grid), kDcCombineThreads, 0, st>>>(p, s, p.batch);
-  }
+  void *args[] = {&p, &s, &mq, &mkv};
+  MXFA_CUDA(cudaLaunchKernel(k, dim3(s.grid), dim3(threads), args, kDcSmemBytes, st));
+  const int cg = combine_grid(p.batch, kDcDv, s.grid);
+  if (dt == MXFA_BF16)
+    decode_combine_kernel<__nv_bfloat16, kDcDv><<<cg, kDcCombineThreads, 0, st>>>(p, s, p.batch);
+  else
+    decode_combine_kernel<__half, kDcDv><<<cg, kDcCombineThreads, 0, st>>>(p, s, p.batch);
   MXFA_CUDA(cudaGetLastError());
   return MXFA_OK;
 }
@@ -652,6 +675,56 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
     return launch_decode_gqa(p, s, dtype, total_kv, kGqKeys, st);
   }
   return launch_simt_any(dtype, p, max_q_len, st);
+}
+
+size_t mxfa_attn_decode_mla_fp8kv_workspace_size(int batch, int max_q_len, int Hq, int max_kv_len, int num_splits) {
+  if (batch <= 0 || Hq <= 0 || num_splits < 0 || (int64_t)max_q_len * Hq > kDcRows) return sizeof(WsHeader);
+  return decode_ws(batch, max_kv_len, num_splits, kDcDv, kDcKeys).total;
+}
+
+mxfa_status_t mxfa_attn_decode_mla_fp8kv(const void *q, const void *kv, float kv_scale, void *o, float *lse,
+                                         const int32_t *qo_indptr, const int32_t *kv_indptr, int batch, int total_q,
+                                         int total_kv, int max_q_len, int max_kv_len, int Hq, int64_t kv_row_stride,
+                                         float softmax_scale, int causal, int num_splits, void *workspace,
+                                         size_t workspace_bytes, void *stream) {
+  if (batch < 0 || total_q < 0 || total_kv < 0 || max_q_len < 0 || max_kv_len < 0 || num_splits < 0)
+    return fail(MXFA_ERR_INVALID_ARG, "negative size");
+  if (Hq <= 0) return fail(MXFA_ERR_INVALID_ARG, "Hq must be positive (Hq=%d)", Hq);
+  if (std::isinf(softmax_scale)) return fail(MXFA_ERR_INVALID_ARG, "softmax_scale is infinite");
+  if (!std::isfinite(kv_scale)) return fail(MXFA_ERR_INVALID_ARG, "kv_scale is not finite");
+  if ((int64_t)max_q_len * Hq > kDcRows)
+    return fail(MXFA_ERR_UNSUPPORTED, "max_q_len * Hq = %lld exceeds %d query rows per sequence",
+                (long long)max_q_len * Hq, kDcRows);
+  if (batch == 0 || total_q == 0) return MXFA_OK;
+  if (!qo_indptr || !kv_indptr) return fail(MXFA_ERR_INVALID_ARG, "qo_indptr / kv_indptr is NULL");
+  if (max_q_len > total_q || max_kv_len > total_kv)
+    return fail(MXFA_ERR_INVALID_ARG, "max length exceeds the total count");
+  MXFA_TRY(check_ptr(q, "q"));
+  MXFA_TRY(check_ptr(o, "o"));
+  MXFA_TRY(check_ptr(lse, "lse", true));
+  MXFA_TRY(check_ptr(kv, "kv"));
+  MXFA_TRY(check_stride(kv_row_stride, 1, "kv_row_stride"));
+  if (kv_row_stride < kDcDqk) return fail(MXFA_ERR_INVALID_ARG, "kv_row_stride is smaller than a row (576 bytes)");
+  MXFA_TRY(check_workspace(workspace, workspace_bytes,
+                           mxfa_attn_decode_mla_fp8kv_workspace_size(batch, max_q_len, Hq, max_kv_len, num_splits)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (strict_mode()) {
+    MXFA_TRY(strict_check_cu(qo_indptr, batch, total_q, max_q_len, "qo_indptr", st));
+    MXFA_TRY(strict_check_cu(kv_indptr, batch, total_kv, max_kv_len, "kv_indptr", st));
+  }
+  AttnParams p{};
+  p.q = q; p.k = kv; p.v = kv; p.o = o; p.lse = lse;
+  p.cu_q = qo_indptr; p.cu_k = kv_indptr;
+  p.batch = batch; p.max_sq = max_q_len; p.max_sk = max_kv_len;
+  p.hq = Hq; p.hkv = 1; p.dqk = kDcDqk; p.dv = kDcDv;
+  p.q_rs = (int64_t)Hq * kDcDqk; p.q_hs = kDcDqk; p.k_rs = kv_row_stride; p.k_hs = kDcDqk;
+  p.v_rs = kv_row_stride; p.v_hs = kDcDv; p.o_rs = (int64_t)Hq * kDcDv; p.o_hs = kDcDv;
+  // s = softmax_scale * <q, kv_scale * code>: the dequantisation scale joins the score scale
+  p.scale_log2 = resolve_scale(softmax_scale, kDcDqk) * kv_scale * kLog2e;
+  p.causal = causal ? 1 : 0;
+  p.hdr = static_cast<WsHeader *>(workspace);
+  p.pairs = nullptr;
+  return launch_decode_tc(p, MXFA_BF16, total_q, total_kv, num_splits, workspace, st, true, kv_scale);
 }
 
 size_t mxfa_attn_decode_kvcache_workspace_size(int batch, int Sq, int Hq, int Hkv, int D, int max_len,

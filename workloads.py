@@ -52,6 +52,7 @@ class Problem:
     batched: bool = False
     mla: bool = False
     kv: torch.Tensor | None = None  # MLA: the single [total_k, 576] cache
+    kv_scale: float | None = None  # set: kv holds E4M3 codes (uint8), element = kv_scale * code value
     check_rows: torch.Tensor | None = None  # [n, 2] (token, head) pairs the oracle evaluates
     meta: dict = field(default_factory=dict)
 
@@ -129,6 +130,29 @@ def mla_decode(seed: int, batch: int, q_len: int, kv_len: int, heads: int = 16, 
                    meta={"batch": batch, "q_len": q_len, "kv_len": kv_len})
 
 
+def mla_decode_fp8(seed: int, batch: int, q_len: int, kv_len: int, heads: int = 16,
+                   lens_kv: list[int] | None = None, causal: bool = False,
+                   name: str = "mla_decode_fp8") -> Problem:
+    """MLA decode over an E4M3 latent cache: q [batch*q_len, heads, 576] bf16;
+    kv [total_kv, 576] E4M3 codes (uint8) with one fp32 scale.  Recipe: q as
+    in ``mla_decode``; the cache is drawn as N(0, 1) fp32 values x (after q,
+    from the same generator), the scale is the fp32 value of max|x| / 448 (the
+    codes then span the format's range, 448 being its largest finite value),
+    and the codes are torch's round-to-nearest-even cast of x / scale, clamped
+    to [-448, 448], to float8_e4m3fn."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    lens_kv = [kv_len] * batch if lens_kv is None else lens_kv
+    tk = sum(lens_kv)
+    q = _randn(g, (batch * q_len, heads, 576), "bf16")
+    x = torch.randn((tk, 576), dtype=torch.float32, generator=g)
+    amax = float(x.abs().max()) if tk else 448.0
+    scale = float(torch.tensor(amax / 448.0, dtype=torch.float32))
+    codes = (x / scale).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    return Problem(name, "bf16", q, codes.view(tk, 1, 576), codes[:, :512].view(tk, 1, 512),
+                   _cu([q_len] * batch), _cu(lens_kv), heads, 1, 576, 512, causal, 576 ** -0.5, mla=True,
+                   kv=codes, kv_scale=scale, meta={"batch": batch, "q_len": q_len, "kv_len": kv_len})
+
+
 def gqa_decode(seed: int, batch: int, q_len: int, kv_len: int, hq: int = 32, hkv: int = 4, d: int = 128,
                dtype: str = "bf16", causal: bool = False, lens_kv: list[int] | None = None,
                name: str | None = None) -> Problem:
@@ -179,6 +203,11 @@ def cfg_varlen_gqa() -> Problem:
 def cfg_mla_decode() -> Problem:
     """MLA split-KV decode, bf16: batch 128, q_len 4, 16 heads, 576/512, kv_len 8192; seed 3."""
     return mla_decode(3, 128, 4, 8192, name="mla_decode_b128_q4_h16_kv8192_bf16")
+
+
+def cfg_mla_decode_fp8() -> Problem:
+    """The same MLA decode shape over an E4M3 cache (bf16 q and output); seed 3."""
+    return mla_decode_fp8(3, 128, 4, 8192, name="mla_decode_b128_q4_h16_kv8192_fp8kv")
 
 
 def kvcache(seed: int, batch: int, Sq: int, Snew: int, seqlens: list[int], hq: int = 32, hkv: int = 4,
