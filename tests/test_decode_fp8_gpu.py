@@ -112,3 +112,43 @@ def test_fp8_rejects_unsupported_shapes():
     with pytest.raises(mx.MxfaError) as e:
         run(p, d, "decode")
     assert e.value.status == mx.MXFA_ERR_UNSUPPORTED
+
+
+def test_fp8_padded_cache_rows():
+    """Cache rows 640 bytes apart (576 codes + padding): the row stride is an
+    argument, and the padding is never read."""
+    import tiled_attention_21_b200 as mx
+    p = workloads.mla_decode_fp8(49, batch=3, q_len=4, kv_len=0, lens_kv=[700, 65, 1300])
+    d = to_dev(p)
+    padded = torch.full((p.total_k, 640), 0x7E, dtype=torch.uint8, device="cuda")  # padding: 448
+    padded[:, :576] = d["kv"]
+    o, l = mx.mxfa_attn_decode_mla_fp8kv(d["q"], padded[:, :576], p.kv_scale, d["cu_q"], d["cu_k"], 4, 1300,
+                                         softmax_scale=p.scale)
+    torch.cuda.synchronize()
+    ro, rl = oracle.problem(p)
+    compare(o, l, ro, rl, p.q.dtype, p.name)
+
+
+def test_fp8_all_sequences_empty():
+    """total_kv = 0 with a valid, never-read cache pointer (the C entry point
+    directly: torch hands out no pointer for an empty tensor): O = 0 and
+    LSE = -inf."""
+    import tiled_attention_21_b200 as mx
+    lib = mx.load()
+    q = torch.randn(8, 16, 576, device="cuda").to(torch.bfloat16)
+    cu_q = torch.tensor([0, 4, 8], dtype=torch.int32, device="cuda")
+    cu_k = torch.zeros(3, dtype=torch.int32, device="cuda")
+    kv = torch.zeros(1, 576, dtype=torch.uint8, device="cuda")
+    o = torch.full((8, 16, 512), 7.0, dtype=torch.bfloat16, device="cuda")
+    l = torch.zeros(8, 16, dtype=torch.float32, device="cuda")
+    need = lib.mxfa_attn_decode_mla_fp8kv_workspace_size(2, 4, 16, 0, 0)
+    ws = mx.workspace(need, q.device)
+    wp, wn = mx._ws_view(ws)
+    st = lib.mxfa_attn_decode_mla_fp8kv(q.data_ptr(), kv.data_ptr(), 0.5, o.data_ptr(), l.data_ptr(),
+                                        cu_q.data_ptr(), cu_k.data_ptr(), 2, 8, 0, 4, 0, 16, 576, float("nan"), 0, 0,
+                                        wp, wn, mx._stream(None))
+    assert st == mx.MXFA_OK, lib.mxfa_last_error()
+    torch.cuda.synchronize()
+    assert mx.read_device_status()[0] == 0
+    assert torch.equal(o.float().cpu(), torch.zeros(8, 16, 512))
+    assert bool(torch.isinf(l).all() and (l < 0).all())
