@@ -120,7 +120,7 @@ struct DecodeCtrl {
   uint64_t q_ready;
   uint64_t tile_full[kDcRingTiles], tile_empty[kDcRingTiles];
   uint64_t stage_full[kDcRingTiles];  // fp8 KV: the slot's codes have landed
-  uint64_t low_full[kDcRingTiles];    // fp8 KV: bf16 chunks 0-3 of the slot are written
+  uint64_t low_full[kDcRingTiles];    // fp8 KV: bf16 chunks 0-2 of the slot are written
   uint64_t s_full, s_free, p_full, o_done, o_empty;
   uint64_t drain;
   uint32_t tmem_base;
@@ -462,16 +462,20 @@ __device__ void dc_zero_rows(const AttnParams &p, const DecodeSched &s, int v) {
 // fp8 KV (OCP 8-bit floating point, E4M3: sign, 4 exponent bits with bias 7,
 // 3 mantissa bits, subnormals, no infinities).  A tile's codes (nine
 // unswizzled 64 keys x 64-byte column chunks, 36,864 bytes) land by TMA in
-// the upper half of the ring slot that will hold the tile in bf16; a
-// widening warpgroup turns them in place into the nine 64 x 128-byte,
+// the upper half of the ring slot that will hold the tile in bf16; six
+// widening warps turn them in place into the nine 64 x 128-byte,
 // 128B-swizzled bf16 chunks the MMA reads.  The bf16 chunks 0-3 end below
-// the codes; chunks 4-8 overwrite codes, so those are read into registers
-// before any of them is written.
+// the codes; chunks 4-8 overwrite codes, so every code is read into
+// registers before any of those is written.
 constexpr int kDcStageChunkBytes = kDcKeys * 64;
 constexpr int kDcStageBytes = kDcChunks * kDcStageChunkBytes;  // 36,864
 constexpr int kDcStageOff = kDcChunks * kDcChunkBytes - kDcStageBytes;  // codes: upper half of the slot
 static_assert(4 * kDcChunkBytes <= kDcStageOff, "bf16 chunks 0-3 end below the staged codes");
-constexpr int kDcThreadsFp8 = 384;  // + warps 8-11: the widening warpgroup
+constexpr int kDcThreadsFp8 = 384;  // + warps 8-11, which widen together with warps 2-3
+constexpr int kDcWiden = 192;       // widening threads: warps 8-11, then 2-3
+constexpr int kDcWidenLow = 3;      // bf16 chunks 0-2 are signalled before chunks 3-8
+static_assert((kDcChunks * kDcKeys * 4) % kDcWiden == 0 && (kDcWidenLow * kDcKeys * 4) % kDcWiden == 0,
+              "widening groups divide evenly");
 
 // Four E4M3 codes (the bytes of w, lowest first) to four bf16 values, exactly.
 // Code byte c becomes the 16-bit pattern sign(c) << 15 | (c & 0x7f) << 4: the
@@ -492,8 +496,8 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t &lo, uint3
 }
 
 // FP8 = true: the KV cache holds E4M3 codes (tm_kv is a byte map, box 64 x 64,
-// no swizzle), staged in the ring slots and widened there by warps 8-11 (384
-// threads); from there the MMA and softmax roles run unchanged.  The
+// no swizzle), staged in the ring slots and widened there by warps 8-11 and
+// 2-3 (384 threads); from there the MMA and softmax roles run unchanged.  The
 // dequantisation scale multiplies the scores (through p.scale_log2) and the
 // outputs (s.o_scale).
 template <bool BF16, bool FP8 = false>
@@ -522,10 +526,10 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
   if (threadIdx.x == 0) {
     mbar_init(b_qr, 128);
     for (int x = 0; x < RT; ++x) {
-      mbar_init(b_tf(x), FP8 ? 128 : 1);  // fp8: the 128 widening threads arrive
+      mbar_init(b_tf(x), FP8 ? kDcWiden : 1);  // fp8: the widening threads arrive
       mbar_init(b_te(x), 1);
       mbar_init(b_gf(x), 1);
-      mbar_init(b_lf(x), 128);
+      mbar_init(b_lf(x), kDcWiden);
     }
     mbar_init(b_sf, 1);
     mbar_init(b_sx, 128);
@@ -639,20 +643,20 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
                   k_lo + (uint32_t)((c * kDcChunkBytes + kk * 32) >> 4), k_hi, idesc_s, (c >= 3 || kk > 0) ? 1u : 0u);
         };
         if (FP8) {
-          // chunks 0-3 as soon as they are widened, then 4-8 (the first MMA
+          // chunks 0-2 as soon as they are widened, then 3-8 (the first MMA
           // into each chain, c = 0, 1, 2 at kk = 0, still comes first)
           if (!wait_warp(b_lf(x), (t / RT) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) mma_chunk(c, kk);
+            for (int c = 0; c < kDcWidenLow; ++c) mma_chunk(c, kk);
           if (!wait_warp(b_tf(x), (t / RT) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-            for (int c = 4; c < kDcChunks; ++c) mma_chunk(c, kk);
+            for (int c = kDcWidenLow; c < kDcChunks; ++c) mma_chunk(c, kk);
         } else {
           if (!wait_warp(b_tf(x), (t / RT) & 1, abort_flag, hdr, kDSiteSlotFull)) return false;
           tc_fence_after();
@@ -706,15 +710,16 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < kWaitBudgetNs) {
       }
     }
-  } else if (FP8 && warp >= 8) {
-    // ------------------------------------------------------------ fp8 -> bf16 widening (warps 8-11)
+  } else if (FP8 && (warp >= 8 || warp == 2 || warp == 3)) {
+    // ------------------------------------------------------------ fp8 -> bf16 widening (warps 8-11, 2-3)
     // Per tile 2,304 groups of 16 codes g = (chunk c, key row, u) = 256c +
     // 4 row + u: columns 16u..16u+15 of key `row` in chunk c, which become
     // 16-byte units 2u and 2u+1 of that row of bf16 chunk c, placed by the
-    // 128B swizzle (unit ^ (row & 7)).  Thread t takes groups t + 128i:
-    // eight consecutive threads read 128 contiguous bytes and write eight
-    // distinct units of two rows, so neither side has bank conflicts.
-    const int t = threadIdx.x - 256;
+    // 128B swizzle (unit ^ (row & 7)).  Widening thread t (0-191) takes
+    // groups t + 192i: eight consecutive threads read 128 contiguous bytes
+    // and write eight distinct units of two rows, so neither side has bank
+    // conflicts.
+    const int t = warp >= 8 ? threadIdx.x - 256 : threadIdx.x + 64;
     uint8_t *ring = smem_raw + (ring_u32 - smem_u32(smem_raw));
     auto put = [&](uint8_t *slot, int g, const uint4 &w) {
       const int c = g >> 8, row = (g >> 2) & 63, u = g & 3;
@@ -727,20 +732,22 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       *reinterpret_cast<uint4 *>(drow + (((2 * u) ^ (row & 7)) << 4)) = a;
       *reinterpret_cast<uint4 *>(drow + (((2 * u + 1) ^ (row & 7)) << 4)) = b;
     };
+    constexpr int kLow = kDcWidenLow * kDcKeys * 4 / kDcWiden;                   // groups per thread, chunks 0-2
+    constexpr int kHigh = (kDcChunks - kDcWidenLow) * kDcKeys * 4 / kDcWiden;  // chunks 3-8
     uint32_t tc = 0;
     bool ok = true;
     for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
       const int4 sd = dc_seg(p, s, sg);
       for (int j = sd.y; j < sd.z; ++j, ++tc) {
         const int y = tc % RT;
-        // The four warps give up together (an AND over the warpgroup), so
-        // none of them is left waiting at the named barrier below.
+        // The six warps give up together (an AND over the widening threads),
+        // so none of them is left waiting at the named barrier below.
         const uint32_t got = wait_bar(b_gf(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull) ? 1u : 0u;
         uint32_t all;
         asm volatile(
-            "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+            "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
             : "=r"(all)
-            : "r"(got)
+            : "r"(got), "n"(kDcWiden)
             : "memory");
         if (!all) {
           ok = false;
@@ -748,19 +755,20 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         }
         uint8_t *slot = ring + y * kDcChunks * kDcChunkBytes;
         const uint4 *codes = reinterpret_cast<const uint4 *>(slot + kDcStageOff);  // group g at codes[g]
-        // chunks 0-3 (groups 0-1023): their bf16 rows end below the codes
-#pragma unroll 4
-        for (int i = 0; i < 8; ++i) put(slot, t + 128 * i, codes[t + 128 * i]);
+        // chunks 0-2: their bf16 rows end below the codes
+#pragma unroll
+        for (int i = 0; i < kLow; ++i) put(slot, t + kDcWiden * i, codes[t + kDcWiden * i]);
         fence_proxy_async_smem();
-        mbar_arrive(b_lf(y));  // S may start on chunks 0-3
-        // chunks 4-8 (groups 1024-2303) overwrite codes: every thread reads
-        // its groups (and has read its chunk 0-3 groups) before any write
-        uint4 w[10];
+        mbar_arrive(b_lf(y));  // S may start on chunks 0-2
+        // chunks 3-8 (from chunk 4 on) overwrite codes: every thread reads
+        // its groups (and has read its chunk 0-2 groups) before any write
+        constexpr int g0 = kDcWidenLow * kDcKeys * 4;
+        uint4 w[kHigh];
 #pragma unroll
-        for (int i = 0; i < 10; ++i) w[i] = codes[1024 + t + 128 * i];
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int i = 0; i < kHigh; ++i) w[i] = codes[g0 + t + kDcWiden * i];
+        asm volatile("bar.sync 1, %0;" ::"n"(kDcWiden) : "memory");
 #pragma unroll
-        for (int i = 0; i < 10; ++i) put(slot, 1024 + t + 128 * i, w[i]);
+        for (int i = 0; i < kHigh; ++i) put(slot, g0 + t + kDcWiden * i, w[i]);
         fence_proxy_async_smem();  // the MMA reads the chunks through the async proxy
         mbar_arrive(b_tf(y));
       }
