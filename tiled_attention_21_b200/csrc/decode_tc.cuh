@@ -71,6 +71,10 @@ struct DecodeSched {
   float2 *part_ml; // [max_segs][64] (running max in log2 units, running sum)
   int max_segs;
   int num_splits;  // 0 = automatic
+  // Automatic schedule: whole sequences are kept while the longest CTA of
+  // that deal is within whole_pct % of the even cut (a split piece costs a
+  // partial of 64 rows x Dv fp32 written and re-read, and a combine pass).
+  int whole_pct;
   int grid;
   // KV-cache mode (p.cu_k == nullptr): batch entry b has cache_seqlens[b] + add
   // keys; key position pos is cache row b*page_size + pos (dense cache,
@@ -192,8 +196,9 @@ __device__ __forceinline__ int dc_lower_bound(const int4 *segs, int n, int x) {
 //   pieces       = num_splits > 0: min(k, n_b) near-equal pieces per sequence;
 //                  automatic: whole sequences, unless cutting the global tile
 //                  sequence at the CTA boundaries c*T/G shortens the longest
-//                  CTA by more than a fifth (splitting costs partial writes,
-//                  a combine pass and an extra Q load per piece).
+//                  CTA by more than DecodeSched::whole_pct allows (splitting
+//                  costs partial writes, a combine pass and an extra Q load
+//                  per piece).
 __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, DecodeSched s) {
   using Scan = cub::BlockScan<int, 1024>;
   __shared__ typename Scan::TempStorage tmp;
@@ -234,7 +239,7 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     // longest CTA with whole sequences (they are dealt out by first tile) vs. the even cut
     const int64_t whole = (int64_t)max_n * ((B + G - 1) / G);
     const int64_t even = (T + G - 1) / G;
-    split_mode = (s.num_splits > 0) ? 1 : (5 * whole > 6 * even ? 2 : 0);  // 0 whole, 1 k pieces, 2 even cut
+    split_mode = (s.num_splits > 0) ? 1 : (100 * whole > s.whole_pct * even ? 2 : 0);  // 0 whole, 1 k pieces, 2 even cut
   }
   __syncthreads();
   {
