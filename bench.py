@@ -406,6 +406,8 @@ def main():
                       "algorithmic_bytes": fbytes, "l2": "inputs (604 MB of codes) larger than L2",
                       "kv_rows_per_s": pf.total_k * world / (fms / 1e3),
                       "mma_tflops": fflops / (fms / 1e3) / 1e12,
+                      "limit": "not HBM: the same M = 64 bf16 MMAs per KV row as the bf16 cache, plus the "
+                               "shared-memory traffic of widening the codes; compare kv_rows_per_s with decode's",
                       "roofline": {"bound": "hbm", "achieved": fgbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                                    "frac": fgbs / pk["hbm_gbs"],
                                    "traffic": recorded_traffic("decode", pf.name),
