@@ -150,14 +150,21 @@ class ClockSampler:
 
 
 def dist_setup(n):
+    """One process per GPU (RANK / WORLD_SIZE / LOCAL_RANK / MASTER_* from the
+    launcher).  The data path has no collective: the process group carries
+    only the timing barrier and the max over ranks.  NCCL on GPUs; gloo on a
+    host without one (the multi-process tests)."""
     if n <= 1 and "RANK" not in os.environ:
         return 0, 1, 0
     import torch.distributed as dist
     rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
     local = int(os.environ.get("LOCAL_RANK", rank))
-    torch.cuda.set_device(local)
     from datetime import timedelta
-    dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        dist.init_process_group("gloo", timeout=timedelta(seconds=120))
     return rank, world, local
 
 
@@ -171,9 +178,17 @@ def max_over_ranks(x, world):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return t.item()
+
+
+def job_rate(units_per_step, steps, world, t_ms):
+    """Whole-job throughput of `world` replicas that each process
+    `units_per_step` per step: all ranks' units over the slowest rank's time
+    (`t_ms`, the max over ranks of the timed steps)."""
+    return units_per_step * steps * world / (t_ms / 1e3)
 
 
 def time_steps(fn, steps, warmup, flush, stream, world):
@@ -300,7 +315,7 @@ def main():
         raise RuntimeError(f"device status {st} at site 0x{site:x}")
     t_ms = max_over_ranks(sum(times), world) if times else float("nan")
     ms_per_step = t_ms / max(1, args.steps)
-    value = flops * args.steps * world / (t_ms / 1e3) / 1e12 if times else float("nan")
+    value = job_rate(flops, args.steps, world, t_ms) / 1e12 if times else float("nan")
     kern_ms = statistics.mean(times) if times else float("nan")  # one kernel launch per step
     achieved = flops / (kern_ms / 1e3) / 1e12
     traffic = recorded_traffic("attn_fwd_tc_kernel", "batched_causal_b4_h16_s2048_d128_bf16")
