@@ -105,6 +105,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
 
   // This CTA's pieces: those whose first tile lies in its tile range (or,
   // in the single-launch schedule, piece blockIdx.x if it exists).
+  dc_pdl_wait();  // the schedule kernel's output (a no-op in the single launch)
   int seg_lo, seg_hi;
   if (s.arith_k > 0) {
     seg_lo = blockIdx.x;
@@ -420,6 +421,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     }
   }
 
+  dc_pdl_release();  // this CTA's pieces are done: the combine kernel may launch
   __syncwarp();
   __syncthreads();
   if (warp == 1) {

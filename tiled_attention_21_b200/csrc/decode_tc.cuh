@@ -138,6 +138,15 @@ enum : uint32_t {
 
 __device__ __forceinline__ int dc_range_start(int c, int T, int G) { return (int)(((int64_t)c * T) / G); }
 
+// Programmatic dependent launch.  The decode kernel (after the schedule
+// kernel) and the combine kernel (after the decode kernel) are launched with
+// programmatic stream serialisation, so their CTAs may become resident while
+// the kernel before them still runs: dc_pdl_wait() blocks until that kernel
+// has completed and its writes are visible, and dc_pdl_release() lets the
+// next kernel's CTAs launch.  Without such a dependency both are no-ops.
+__device__ __forceinline__ void dc_pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void dc_pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Four outputs, rounded to the 16-bit output type, as one 8-byte store.
 template <typename T>
 __device__ __forceinline__ void dc_store4(T *dst, float a, float b, float c, float d) {
@@ -200,6 +209,7 @@ __device__ __forceinline__ int dc_lower_bound(const int4 *segs, int n, int x) {
 //                  costs partial writes, a combine pass and an extra Q load
 //                  per piece).
 __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, DecodeSched s) {
+  dc_pdl_release();  // the decode kernel's CTAs may set up while this runs
   using Scan = cub::BlockScan<int, 1024>;
   __shared__ typename Scan::TempStorage tmp;
   __shared__ int carry, max_n, split_mode;
@@ -557,6 +567,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
 
   // This CTA's pieces: those whose first tile lies in its tile range (or,
   // in the single-launch schedule, piece blockIdx.x if it exists).
+  dc_pdl_wait();  // the schedule kernel's output (a no-op in the single launch)
   int seg_lo, seg_hi;
   if (s.arith_k > 0) {
     seg_lo = blockIdx.x;
@@ -969,6 +980,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     }
   }
 
+  dc_pdl_release();  // this CTA's pieces are done: the combine kernel may launch
   __syncwarp();
   __syncthreads();
   if (warp == 1) {
@@ -998,6 +1010,7 @@ constexpr int kDcCombineThreads = 256;
 template <typename T, int DV>
 __global__ void __launch_bounds__(kDcCombineThreads) decode_combine_kernel(const AttnParams p, const DecodeSched s,
                                                                            int n_seq) {
+  dc_pdl_wait();  // the decode kernel's partials
   constexpr int kBlocks = DV / 16;  // 16-column blocks per row
   const int r = threadIdx.x % kDcRows, q = threadIdx.x / kDcRows;
   const int n_items = n_seq * kBlocks;

@@ -320,6 +320,25 @@ mxfa_status_t prefill(AttnParams &p, mxfa_dtype_t dt, int D, bool varlen, int64_
   return bf ? launch_tc<64, true>(p, mq, mk, mv, st) : launch_tc<64, false>(p, mq, mk, mv, st);
 }
 
+// Launch with programmatic stream serialisation: the kernel's CTAs may start
+// while the preceding kernel in the stream still runs; the kernel calls
+// dc_pdl_wait() before it reads that kernel's results.
+mxfa_status_t launch_dependent(const void *kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                               void **args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  MXFA_CUDA(cudaLaunchKernelExC(&cfg, kernel, args));
+  return MXFA_OK;
+}
+
 // Workspace layout of the tensor-core decode kernels: `batch` decode
 // sequences (batch entries x KV heads that form separate sequences), Dv
 // output columns.
@@ -423,11 +442,15 @@ mxfa_status_t launch_decode_gqa_t(AttnParams &p, const DecodeSched &s, mxfa_dtyp
   decode_prep_kernel<<<1, 1024, 0, st>>>(p, s);
   MXFA_CUDA(cudaGetLastError());
   MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(k), GqaCfg<D>::kSmemBytes));
-  k<<<s.grid, kGqThreads, GqaCfg<D>::kSmemBytes, st>>>(p, s, mk, mv);
-  MXFA_CUDA(cudaGetLastError());
+  DecodeSched sd = s;
+  int ns = n_seq;
+  void *args[] = {&p, &sd, &mk, &mv};
+  MXFA_TRY(launch_dependent(reinterpret_cast<const void *>(k), dim3(s.grid), dim3(kGqThreads), GqaCfg<D>::kSmemBytes,
+                            st, args));
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  decode_combine_kernel<T, D><<<combine_grid(n_seq, D, s.grid), kDcCombineThreads, 0, st>>>(p, s, n_seq);
-  MXFA_CUDA(cudaGetLastError());
+  void *cargs[] = {&p, &sd, &ns};
+  MXFA_TRY(launch_dependent(reinterpret_cast<const void *>(decode_combine_kernel<T, D>),
+                            dim3(combine_grid(n_seq, D, s.grid)), dim3(kDcCombineThreads), 0, st, cargs));
   return MXFA_OK;
 }
 
@@ -476,13 +499,13 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
   decode_prep_kernel<<<1, 1024, 0, st>>>(p, s);
   MXFA_CUDA(cudaGetLastError());
   void *args[] = {&p, &s, &mq, &mkv};
-  MXFA_CUDA(cudaLaunchKernel(k, dim3(s.grid), dim3(threads), args, kDcSmemBytes, st));
+  MXFA_TRY(launch_dependent(k, dim3(s.grid), dim3(threads), kDcSmemBytes, st, args));
   const int cg = combine_grid(p.batch, kDcDv, s.grid);
-  if (dt == MXFA_BF16)
-    decode_combine_kernel<__nv_bfloat16, kDcDv><<<cg, kDcCombineThreads, 0, st>>>(p, s, p.batch);
-  else
-    decode_combine_kernel<__half, kDcDv><<<cg, kDcCombineThreads, 0, st>>>(p, s, p.batch);
-  MXFA_CUDA(cudaGetLastError());
+  int ns = p.batch;
+  void *cargs[] = {&p, &s, &ns};
+  const void *ck = dt == MXFA_BF16 ? reinterpret_cast<const void *>(decode_combine_kernel<__nv_bfloat16, kDcDv>)
+                                   : reinterpret_cast<const void *>(decode_combine_kernel<__half, kDcDv>);
+  MXFA_TRY(launch_dependent(ck, dim3(cg), dim3(kDcCombineThreads), 0, st, cargs));
   return MXFA_OK;
 }
 
