@@ -93,6 +93,10 @@ struct DecodeSched {
   // counts the pieces that have stored theirs (zeroed before the launch).
   int arith_k;
   int *sync;
+  // Schedule kernel output: the number of sequences not stored directly by
+  // the decode kernel (split into pieces, or with no piece at all); the
+  // combine kernel has nothing to do when it is 0.
+  int *n_multi;
   // Factor of every stored output and partial accumulator: 1, or the KV
   // dequantisation scale of the fp8-KV MLA kernel (the scores' share of that
   // scale is folded into AttnParams::scale_log2 by the host).
@@ -212,13 +216,14 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
   dc_pdl_release();  // the decode kernel's CTAs may set up while this runs
   using Scan = cub::BlockScan<int, 1024>;
   __shared__ typename Scan::TempStorage tmp;
-  __shared__ int carry, max_n, split_mode;
+  __shared__ int carry, max_n, split_mode, n_multi;
   __shared__ int cut[kDcMaxGrid + 1];  // x_c = c*T/G, c = 0..G
   __shared__ int ps[kDcMaxGrid + 1];   // ps[c]: c' in [1, c] with cut[c'] != cut[c'-1] (distinct cut values)
   const int tid = threadIdx.x, B = p.batch * s.heads, G = s.grid;
   if (tid == 0) {
     carry = 0;
     max_n = 0;
+    n_multi = 0;
   }
   __syncthreads();
   for (int base = 0; base < B; base += 1024) {
@@ -292,6 +297,7 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     const int b = base + tid;
     const int k = b < B ? pieces(b) : 0;
     if (b < B) s.seg_cnt[b] = k;
+    if (b < B && k != 1) atomicAdd(&n_multi, 1);
     int incl, total;
     Scan(tmp).InclusiveSum(k, incl, total);
     if (b < B) s.seg_base[b] = carry + incl - k;
@@ -342,6 +348,7 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
   if (tid == 0) {
     p.hdr->n_units = (uint32_t)min(n_segs, s.max_segs);
     p.hdr->n_aux = (uint32_t)T;
+    *s.n_multi = n_multi;
     if (n_segs > s.max_segs) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x401);
   }
 }
@@ -1002,25 +1009,30 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
 // ----------------------------------------------------------------------------
 // Merge the pieces of every sequence that was split.  Row r of sequence
 // v = (b, g) is query token r / G of batch entry b, head g*G + r % G, with
-// G = Hq / heads.  Grid-stride over items (sequence v, block of 16 columns);
-// thread (r, q) of the 256 takes row r and columns 4(4j + q) .. +3 of item j,
-// so the partial loads of a warp are contiguous.  An item whose sequence was
-// not split (stored directly by the decode kernel) costs one load.
+// G = Hq / heads.  One thread per (sequence v, 4-column group c4, row r) for
+// r < R = min(64, max_q * G), rows fastest, so a warp's partial loads are
+// contiguous; grid-stride.  Every unit is independent, so the dependent
+// loads of all of them are in flight together.  A unit whose sequence was
+// not split (stored directly by the decode kernel) costs one load, and when
+// no sequence was split or left empty the kernel returns at once.
 constexpr int kDcCombineThreads = 256;
 template <typename T, int DV>
 __global__ void __launch_bounds__(kDcCombineThreads) decode_combine_kernel(const AttnParams p, const DecodeSched s,
                                                                            int n_seq) {
   dc_pdl_wait();  // the decode kernel's partials
-  constexpr int kBlocks = DV / 16;  // 16-column blocks per row
-  const int r = threadIdx.x % kDcRows, q = threadIdx.x / kDcRows;
-  const int n_items = n_seq * kBlocks;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int v = item / kBlocks, c4 = (item % kBlocks) * 4 + q;
+  if (*reinterpret_cast<volatile int *>(s.n_multi) == 0) return;
+  constexpr int C4 = DV / 4;  // 4-column groups per row
+  const int G = p.hq / s.heads;
+  const int R = min(kDcRows, p.max_sq * G);
+  const int64_t n_units = (int64_t)n_seq * C4 * R;
+  for (int64_t unit = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; unit < n_units;
+       unit += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(unit % R), c4 = (int)((unit / R) % C4), v = (int)(unit / ((int64_t)R * C4));
     const int cnt = s.seg_cnt[v];
     // not split: stored directly by the decode kernel (a sequence with no
     // piece, cnt = 0, is written here: O = 0, LSE = -inf)
     if (cnt == 1) continue;
-    const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
+    const int b = v / s.heads, gh = v % s.heads;
     const int2 qr = dc_q(p, b);
     if (r >= qr.y * G) continue;
     const int base = s.seg_base[v];

@@ -343,7 +343,7 @@ mxfa_status_t launch_dependent(const void *kernel, dim3 grid, dim3 block, size_t
 // sequences (batch entries x KV heads that form separate sequences), Dv
 // output columns.
 struct DecodeWs {
-  size_t n_tiles, tile_pre, seg_base, seg_cnt, kv_len, sync, segs, part_ml, part_acc, total;
+  size_t n_tiles, tile_pre, seg_base, seg_cnt, kv_len, sync, multi, segs, part_ml, part_acc, total;
   int max_segs;
 };
 DecodeWs decode_ws(int batch, int max_kv_len, int num_splits, int dv, int keys) {
@@ -356,7 +356,8 @@ DecodeWs decode_ws(int batch, int max_kv_len, int num_splits, int dv, int keys) 
   w.seg_cnt = w.seg_base + align256(sizeof(int) * (size_t)(batch + 1));
   w.kv_len = w.seg_cnt + align256(sizeof(int) * (size_t)batch);
   w.sync = w.kv_len + align256(sizeof(int) * (size_t)batch);
-  w.segs = w.sync + align256(sizeof(int) * (size_t)batch);
+  w.multi = w.sync + align256(sizeof(int) * (size_t)batch);
+  w.segs = w.multi + align256(sizeof(int));
   w.part_ml = w.segs + align256(sizeof(int4) * (size_t)w.max_segs);
   w.part_acc = w.part_ml + align256(sizeof(float2) * (size_t)w.max_segs * kDcRows);
   w.total = w.part_acc + align256(sizeof(float) * (size_t)w.max_segs * kDcRows * dv);
@@ -393,6 +394,7 @@ DecodeSched decode_sched(const AttnParams &p, int heads, int num_splits, int dv,
   s.part_acc = reinterpret_cast<float *>(base + w.part_acc);
   s.kv_len = reinterpret_cast<int *>(base + w.kv_len);
   s.sync = reinterpret_cast<int *>(base + w.sync);
+  s.n_multi = reinterpret_cast<int *>(base + w.multi);
   s.arith_k = 0;
   s.o_scale = 1.f;
   s.max_segs = w.max_segs;
