@@ -171,3 +171,22 @@ def test_kvcache_validation(lib):
     assert c(B=0) == m.MXFA_OK                               # nothing to do
     need = lib.mxfa_attn_decode_kvcache_workspace_size(64, 1, 32, 4, 128, 8192, 0, 2)
     assert need > 256 and need == lib.mxfa_attn_decode_splitkv_workspace_size(64, 1, 32, 4, 128, 8192, 0, 2)
+
+
+def test_fp8_binding_rejects_bad_tensors(lib):
+    """The binding checks dtypes and layouts before any device work."""
+    import torch
+    import tiled_attention_21_b200 as m
+    q = torch.zeros(8, 16, 576, dtype=torch.bfloat16)
+    kv = torch.zeros(64, 576, dtype=torch.uint8)
+    cu = torch.zeros(3, dtype=torch.int32)
+    with pytest.raises(ValueError):  # q must be bf16
+        m.mxfa_attn_decode_mla_fp8kv(q.float(), kv, 1.0, cu, cu, 4, 32)
+    with pytest.raises(ValueError):  # q must be contiguous
+        m.mxfa_attn_decode_mla_fp8kv(q.transpose(0, 1), kv, 1.0, cu, cu, 4, 32)
+    with pytest.raises(ValueError):  # codes are bytes
+        m.mxfa_attn_decode_mla_fp8kv(q, kv.to(torch.int16), 1.0, cu, cu, 4, 32)
+    with pytest.raises(ValueError):  # [total_kv, 576] with unit stride inside a row
+        m.mxfa_attn_decode_mla_fp8kv(q, kv.view(64, 1, 576), 1.0, cu, cu, 4, 32)
+    with pytest.raises(ValueError):
+        m.mxfa_attn_decode_mla_fp8kv(q, kv.t(), 1.0, cu, cu, 4, 32)
