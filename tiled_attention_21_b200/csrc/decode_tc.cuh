@@ -127,7 +127,8 @@ __device__ __forceinline__ int dc_krow(const AttnParams &p, const DecodeSched &s
 struct DecodeCtrl {
   uint64_t q_ready;
   uint64_t tile_full[kDcRingTiles], tile_empty[kDcRingTiles];
-  uint64_t stage_full[kDcRingTiles];  // fp8 KV: the slot's codes have landed
+  uint64_t stage_full[kDcRingTiles];  // fp8 KV: the codes of chunks 0-2 of the slot have landed
+  uint64_t stage_rest[kDcRingTiles];  // fp8 KV: the codes of chunks 3-8 have landed
   uint64_t low_full[kDcRingTiles];    // fp8 KV: bf16 chunks 0-2 of the slot are written
   uint64_t s_full, s_free, p_full, o_done, o_empty;
   uint64_t drain;
@@ -541,6 +542,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
   auto b_tf = [&](int x) { return smem_u32(&ctrl->tile_full[x]); };
   auto b_te = [&](int x) { return smem_u32(&ctrl->tile_empty[x]); };
   auto b_gf = [&](int x) { return smem_u32(&ctrl->stage_full[x]); };
+  auto b_gr = [&](int x) { return smem_u32(&ctrl->stage_rest[x]); };
   auto b_lf = [&](int x) { return smem_u32(&ctrl->low_full[x]); };
   const uint32_t b_qr = smem_u32(&ctrl->q_ready), b_sf = smem_u32(&ctrl->s_full), b_sx = smem_u32(&ctrl->s_free);
   const uint32_t b_pf = smem_u32(&ctrl->p_full), b_od = smem_u32(&ctrl->o_done), b_oe = smem_u32(&ctrl->o_empty);
@@ -551,6 +553,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       mbar_init(b_tf(x), FP8 ? kDcWiden : 1);  // fp8: the widening threads arrive
       mbar_init(b_te(x), 1);
       mbar_init(b_gf(x), 1);
+      mbar_init(b_gr(x), 1);
       mbar_init(b_lf(x), kDcWiden);
     }
     mbar_init(b_sf, 1);
@@ -607,11 +610,12 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
             ok = false;
             break;
           }
-          if (FP8) {  // the codes, into the upper half of the slot
-            mbar_arrive_expect_tx(b_gf(x), kDcStageBytes);
+          if (FP8) {  // the codes, into the upper half of the slot: chunks 0-2, then 3-8
+            mbar_arrive_expect_tx(b_gf(x), kDcWidenLow * kDcStageChunkBytes);
+            mbar_arrive_expect_tx(b_gr(x), (kDcChunks - kDcWidenLow) * kDcStageChunkBytes);
             for (int c = 0; c < kDcChunks; ++c)
               tma_load_2d(ring_u32 + x * kDcChunks * kDcChunkBytes + kDcStageOff + c * kDcStageChunkBytes, &tm_kv,
-                          b_gf(x), c * 64, k0 + j * kDcKeys);
+                          c < kDcWidenLow ? b_gf(x) : b_gr(x), c * 64, k0 + j * kDcKeys);
             // Tile j + 2 into L2, so that its load (issued once its slot is
             // free) does not wait on HBM: the widening adds to the time from
             // a free slot to a ready tile, which three slots must cover.
@@ -630,6 +634,8 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         const uint32_t uses = tc / RT + ((uint32_t)x < tc % RT ? 1u : 0u);
         if (uses == 0) continue;
         while (!mbar_test(FP8 ? b_gf(x) : b_tf(x), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        }
+        while (FP8 && !mbar_test(b_gr(x), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
         }
       }
     }
@@ -755,6 +761,17 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       *reinterpret_cast<uint4 *>(drow + (((2 * u) ^ (row & 7)) << 4)) = a;
       *reinterpret_cast<uint4 *>(drow + (((2 * u + 1) ^ (row & 7)) << 4)) = b;
     };
+    // The six warps give up a wait together (an AND over the widening
+    // threads), so none of them is left waiting at a named barrier.
+    auto agree = [&](bool got) {
+      uint32_t all;
+      asm volatile(
+          "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+          : "=r"(all)
+          : "r"(got ? 1u : 0u), "n"(kDcWiden)
+          : "memory");
+      return all != 0;
+    };
     constexpr int kLow = kDcWidenLow * kDcKeys * 4 / kDcWiden;                   // groups per thread, chunks 0-2
     constexpr int kHigh = (kDcChunks - kDcWidenLow) * kDcKeys * 4 / kDcWiden;  // chunks 3-8
     uint32_t tc = 0;
@@ -763,16 +780,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       const int4 sd = dc_seg(p, s, sg);
       for (int j = sd.y; j < sd.z; ++j, ++tc) {
         const int y = tc % RT;
-        // The six warps give up together (an AND over the widening threads),
-        // so none of them is left waiting at the named barrier below.
-        const uint32_t got = wait_bar(b_gf(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull) ? 1u : 0u;
-        uint32_t all;
-        asm volatile(
-            "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-            : "=r"(all)
-            : "r"(got), "n"(kDcWiden)
-            : "memory");
-        if (!all) {
+        if (!agree(wait_bar(b_gf(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull))) {
           ok = false;
           break;
         }
@@ -785,6 +793,10 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         mbar_arrive(b_lf(y));  // S may start on chunks 0-2
         // chunks 3-8 (from chunk 4 on) overwrite codes: every thread reads
         // its groups (and has read its chunk 0-2 groups) before any write
+        if (!agree(wait_bar(b_gr(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull))) {
+          ok = false;
+          break;
+        }
         constexpr int g0 = kDcWidenLow * kDcKeys * 4;
         uint4 w[kHigh];
 #pragma unroll
