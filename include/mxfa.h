@@ -160,8 +160,10 @@ mxfa_status_t mxfa_attn_varlen_fwd_noalloc(const void *q, const void *k, const v
  * (or f32) run on the exact CUDA-core kernel.
  * The workspace size takes Hkv because the grouped-query kernel schedules
  * batch * Hkv decode sequences.
- * num_splits: 0 = automatic (the KV of all sequences is cut into
- *   near-equal pieces, one run per SM); k >= 1 = every sequence's KV is cut
+ * num_splits: 0 = automatic: one run of KV tiles per SM, either whole
+ *   sequences dealt out in order or the KV of all sequences cut into
+ *   near-equal pieces, whichever balances better once the cost of merging a
+ *   split sequence's partials is counted; k >= 1 = every sequence's KV is cut
  *   into k pieces.  The result does not depend on it beyond fp32 rounding.
  * Small problems (the MLA-shaped kernel, num_splits = 0, batch no larger
  *   than the SM count and batch * ceil(max_kv_len / 64) at most four tiles per
