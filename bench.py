@@ -2,19 +2,30 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mxfa|reference]
 
-One step = one attention forward of the batched causal prefill workload
-(bf16, B=4, Hq=Hkv=16, Sq=Sk=2048, D=128, seed 1) through the library's
-tensor-core path; the metric is causal-adjusted TFLOP/s (4*B*H*S^2*D / 2
-per step).  The same run also measures the MLA split-KV decode workload
-(bf16, batch 128, q_len 4, 16 heads, 576/512, kv_len 8192, seed 3) in KV
-GB/s, reported under "decode".  Inputs are synthetic (workloads.py); L2 is
-flushed (a 512 MiB write) before every timed step, outside the timed
-interval.  With --gpus N (under torchrun) every rank runs its own replica
-(no collective on the data path; weak scaling) and the time is the max
-over ranks.
+The headline step is one attention forward of the long-context causal
+prefill (bf16, B=1, Hq=Hkv=32, Sq=Sk=32768, D=128, seed 4), the largest
+workload that fits one GPU, through the library's tensor-core path; the
+metric is causal-adjusted TFLOP/s (4*B*H*S^2*D / 2 per step).  The same run
+measures, each as a sub-object of the one JSON line with its own roofline,
+end-to-end number, oracle CPU baseline and clock record:
+  batched_causal    bf16, B=4, H=16, S=2048, D=128, causal (seed 1)
+  varlen_gqa        bf16 varlen, 16 sequences U[128, 4096] (seed 2),
+                    Hq=32, Hkv=8, D=128, causal; the schedule kernel that
+                    precedes the attention kernel is inside the timed call
+  single_head_fp32  fp32, B=1, H=1, S=128, D=64, non-causal (seed 0): us
+                    per call on the exact CUDA-core kernel
+  decode            MLA split-KV decode, bf16, batch 128, q_len 4, 16 heads,
+                    576/512, kv_len 8192 (seed 3), in KV GB/s
+  decode_gqa        grouped-query decode, q_len 1, Hq 32, Hkv 4, D 128, kv 8192
+  decode_fp8        the MLA decode over an E4M3 cache
+Inputs are synthetic (workloads.py).  L2 is flushed (a 512 MiB write)
+before every timed prefill step, outside the timed interval; the decode
+inputs (0.6-1.2 GB) are larger than L2.  With --gpus N (under torchrun)
+every rank runs its own replica (no collective on the data path; weak
+scaling) and each time is the max over ranks.
 
---impl reference times the fp64 CPU oracle on the host cores on a bounded
-sample of the same workload (the reference arm; there is no reference
+--impl reference times the fp64 CPU oracle on the host cores on bounded
+samples of the headline workload (the reference arm; there is no reference
 library to run).
 """
 from __future__ import annotations
@@ -22,7 +33,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -37,7 +47,7 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 METRIC = "attn fwd TFLOP/s (causal-adjusted) & decode KV GB/s, % of B200 roofline"
-PREFILL_CFG = dict(B=4, H=16, S=2048, D=128)
+HEADLINE = dict(B=1, H=32, S=32768, D=128)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -52,6 +62,12 @@ def peaks():
 def prefill_flops(B, H, S, D, causal=True):
     f = 4.0 * B * H * S * S * D
     return f / 2 if causal else f
+
+
+def varlen_flops(p):
+    """Conventional causal-adjusted work of a varlen problem: 4*Hq*D*L^2/2 per sequence."""
+    f = sum(4.0 * p.hq * p.dqk * L * L for L in p.seqlens_q())
+    return f / 2 if p.causal else f
 
 
 def decode_bytes(p):
@@ -192,7 +208,8 @@ def job_rate(units_per_step, steps, world, t_ms):
 
 
 def time_steps(fn, steps, warmup, flush, stream, world):
-    """Per-step CUDA-event times (ms) on `stream`; L2 flushed before each step."""
+    """Per-step CUDA-event times (ms) on `stream`; `flush` before each step,
+    outside the timed interval."""
     for _ in range(warmup):
         flush()
         fn()
@@ -214,36 +231,96 @@ def time_steps(fn, steps, warmup, flush, stream, world):
     return [a.elapsed_time(b) for a, b in evs]
 
 
-def cpu_baseline_prefill(target_s: float = 12.0):
-    """The fp64 oracle on host cores over a bounded sample of the prefill
-    workload: random (token, head) rows, throughput in causal-adjusted
-    TFLOP/s of the rows evaluated (4*D*visible keys per row)."""
+# ---------------------------------------------------------------- CPU baseline (the oracle, timed)
+def _visible_keys(p, pairs):
+    """Visible keys of each sampled (token, head) row (bottom-right causal)."""
+    cq, ck = p.cu_q.tolist(), p.cu_k.tolist()
+    out = []
+    import bisect
+    for tok in pairs[:, 0].tolist():
+        b = bisect.bisect_right(cq, tok) - 1
+        sq, sk, i = cq[b + 1] - cq[b], ck[b + 1] - ck[b], tok - cq[b]
+        out.append(sk if not p.causal else max(0, min(sk, i + 1 + sk - sq)))
+    return out
+
+
+def _sample_pairs(p, n, seed):
+    """n (token, head) rows of problem p drawn uniformly with a seeded generator."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    tok = torch.randint(0, p.total_q, (n,), generator=g)
+    hd = torch.randint(0, p.hq, (n,), generator=g)
+    return torch.stack([tok, hd], 1)
+
+
+def cpu_baseline(p, kind: str, target_s: float = 8.0, full_units=None):
+    """The fp64 oracle as it stands on the host cores over a bounded random
+    sample of (token, head) rows of workload `p`, scaled to the metric's
+    unit.  kind "flops": TFLOP/s of the contraction work of the rows
+    evaluated, 2*(Dqk+Dv) per visible (query, key) pair (4*D for Dqk = Dv,
+    as in the causal-adjusted metric); kind "bytes": the workload's
+    algorithmic bytes `full_units` in proportion to the rows evaluated, in
+    GB/s."""
     import oracle
-    p = workloads.cfg_batched_causal()
     threads = oracle.default_threads()
-    S, D = PREFILL_CFG["S"], PREFILL_CFG["D"]
+    n_rows = p.total_q * p.hq
 
     def run(n, seed):
-        pairs = workloads.sample_rows(p, max(1, n // p.hq), seed)
-        i_local = pairs[:, 0] % S
-        flops = float((4 * D * (i_local + 1)).sum())
+        pairs = _sample_pairs(p, n, seed)
         t0 = time.perf_counter()
         oracle.problem(p, pairs=pairs, threads=threads)
-        return time.perf_counter() - t0, flops, pairs.shape[0]
+        return time.perf_counter() - t0, pairs
 
-    t, f, n = run(256, 7)
-    n2 = int(max(256, min(200000, n * target_s / max(t, 1e-3))))
-    t, f, n = run(n2, 8)
-    return {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} random (token, head) rows of the B=4 H=16 S=2048 D=128 causal workload "
-                      f"(plus first/last rows), fp64, {t:.1f} s wall"}
+    t, pairs = run(4 * threads, 7)
+    n = int(max(threads, min(n_rows, pairs.shape[0] * target_s / max(t, 1e-3))))
+    t, pairs = run(n, 8)
+    rows = pairs.shape[0]
+    if kind == "flops":
+        work = sum(2.0 * (p.dqk + p.dv) * nv for nv in _visible_keys(p, pairs))
+        value, unit = work / t / 1e12, "TFLOP/s"
+    else:
+        value, unit = full_units * rows / n_rows / t / 1e9, "GB/s"
+    return {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+            "sample": f"{rows} random (token, head) rows of the {n_rows} of {p.name}, fp64, {t:.1f} s wall" +
+                      ("; rate = the workload's algorithmic bytes x rows evaluated / all rows" if kind == "bytes"
+                       else "; work = 2*(Dqk+Dv) per visible (query, key) pair")}
+
+
+def cpu_baseline_full_us(p, target_s: float = 3.0):
+    """The oracle on the whole (small) problem, repeated for about target_s: us per call."""
+    import oracle
+    threads = oracle.default_threads()
+    oracle.problem(p, threads=threads)
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < target_s:
+        oracle.problem(p, threads=threads)
+        n += 1
+    t = time.perf_counter() - t0
+    return {"value": t / n * 1e6, "unit": "us", "cores": threads, "kind": "oracle",
+            "sample": f"the whole problem ({p.total_q * p.hq} rows), {n} calls, fp64, {t:.1f} s wall"}
+
+
+def headline_problem():
+    return workloads.cfg_long_causal(S=HEADLINE["S"], H=HEADLINE["H"])
+
+
+def headline_config(p, flops, world):
+    return headline_config_of(p.name, flops, world)
+
+
+def headline_config_of(name, flops, world):
+    return {"workload": name, "B": HEADLINE["B"], "H": HEADLINE["H"], "seq_len": HEADLINE["S"],
+            "head_dim": HEADLINE["D"], "causal": True, "flops_per_step": flops,
+            "l2": "flushed before every step (512 MiB write); inputs (805 MB q, k, v) are larger than L2",
+            "parallelism": f"replicas x{world}"}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    res = [cpu_baseline_prefill(target_s=max(2.0, 60.0 / max(1, args.steps + args.warmup))) for _ in
-           range(args.warmup + args.steps)]
+    p = headline_problem()
+    flops = prefill_flops(HEADLINE["B"], HEADLINE["H"], HEADLINE["S"], HEADLINE["D"])
+    res = [cpu_baseline(p, "flops", target_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+           for _ in range(args.warmup + args.steps)]
     vals = [r["value"] for r in res[args.warmup:]]
     v = statistics.mean(vals)
     cb = dict(res[-1])
@@ -251,24 +328,265 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "batched_causal_b4_h16_s2048_d128_bf16", "l2": "n/a (host)"},
+            "config": headline_config(p, flops, world) | {"l2": "n/a (host)"},
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- legs
+class Bench:
+    def __init__(self, args, world, local, dev, stream):
+        import tiled_attention_21_b200 as mx
+        self.mx = mx
+        self.args, self.world, self.local, self.dev, self.stream = args, world, local, dev, stream
+        self.flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        self.pk, self.pk_kind = peaks()
+        self.rank0_cpu = world == 1 and not args.no_cpu_baseline
+
+    def flush(self):
+        self.flush_buf.zero_()
+
+    def timed(self, fn, steps, warmup=3, flush=True):
+        """(per-step times, clock summary); the times of the slowest rank."""
+        with ClockSampler(self.local) as clk:
+            times = time_steps(fn, steps, warmup, self.flush if flush else (lambda: None), self.stream,
+                               self.world)
+        return times, clk.summary()
+
+    def check_status(self, ws):
+        st, site = self.mx.read_device_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status {st} at site 0x{site:x}")
+
+    def tensor_roofline(self, flops, kern_ms, kernel, workload):
+        achieved = flops / (kern_ms / 1e3) / 1e12
+        peak = self.pk["bf16_tflops"]
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": recorded_traffic("attn_fwd_tc_kernel", workload), "kernel": kernel,
+                "peak_kind": f"{self.pk_kind} burst dense bf16 (cuBLAS)"}
+
+    def hbm_roofline(self, nbytes, kern_ms, kernel_key, workload):
+        gbs = nbytes / (kern_ms / 1e3) / 1e9
+        peak = self.pk["hbm_gbs"]
+        return {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                "traffic": recorded_traffic(kernel_key, workload), "peak_kind": f"{self.pk_kind} HBM copy"}
+
+    # -------- batched prefill (headline and batched_causal)
+    def batched_prefill(self, p, steps, cpu=True):
+        mx, dev, stream, world = self.mx, self.dev, self.stream, self.world
+        B = p.meta["B"]
+        S, H, D = p.meta["Sq"], p.hq, p.dqk
+        q = p.q.view(B, S, H, D).to(dev)
+        k = p.k.view(B, S, H, D).to(dev)
+        v = p.v.view(B, S, H, D).to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, S, H), dtype=torch.float32, device=dev)
+        ws = mx.workspace(256, dev)
+
+        def step():
+            mx.mxfa_attn_fwd(q, k, v, causal=True, out=o, lse=lse, ws=ws, stream=stream)
+
+        flops = prefill_flops(B, H, S, D)
+        times, clocks = self.timed(step, steps, self.args.warmup)
+        self.check_status(ws)
+        t_ms = max_over_ranks(sum(times), world)
+        kern_ms = max_over_ranks(statistics.mean(times), world)  # one kernel launch per step
+        res = {"workload": p.name, "value": job_rate(flops, steps, world, t_ms) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": t_ms / steps, "steps": steps, "flops_per_step": flops,
+               "roofline": self.tensor_roofline(flops, kern_ms, f"attn_fwd_tc_kernel<{D},bf16>", p.name),
+               "clocks": clocks, "gpu_launches": steps}
+        # end to end through the public API with host buffers
+        hq, hk, hv = (t.view(B, S, H, D).pin_memory() for t in (p.q, p.k, p.v))
+        ho = torch.empty((B, S, H, D), dtype=torch.bfloat16).pin_memory()
+        hl = torch.empty((B, S, H), dtype=torch.float32).pin_memory()
+        dq, dk, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv_.copy_(hv, non_blocking=True)
+            mx.mxfa_attn_fwd(dq, dk, dv_, causal=True, out=o, lse=lse, ws=ws, stream=stream)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        n_e2e = max(5, steps // 3)
+        e2e_times, _ = self.timed(e2e_step, n_e2e, 2)
+        e2e_ms = max_over_ranks(sum(e2e_times), world)
+        res["e2e"] = {"value": job_rate(flops, n_e2e, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
+                      "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4}
+        res["cpu_baseline"] = cpu_baseline(p, "flops") if (cpu and self.rank0_cpu) else None
+        del q, k, v, o, dq, dk, dv_
+        return res
+
+    # -------- varlen prefill (varlen_gqa)
+    def varlen_prefill(self, p, steps):
+        mx, dev, stream, world = self.mx, self.dev, self.stream, self.world
+        d = workloads.to_device(p, dev)
+        o = torch.empty_like(d["q"])
+        lse = torch.empty((p.total_q, p.hq), dtype=torch.float32, device=dev)
+        max_q, max_k = max(p.seqlens_q()), max(p.seqlens_k())
+        ws = mx.workspace(mx.load().mxfa_attn_varlen_fwd_workspace_size(p.batch, max_q, max_k, p.hq, p.dqk, 2), dev)
+
+        def step():
+            mx.mxfa_attn_varlen_fwd(d["q"], d["k"], d["v"], d["cu_q"], d["cu_k"], max_q, max_k, causal=True,
+                                    out=o, lse=lse, ws=ws, stream=stream)
+
+        flops = varlen_flops(p)
+        times, clocks = self.timed(step, steps, self.args.warmup)
+        self.check_status(ws)
+        t_ms = max_over_ranks(sum(times), world)
+        kern_ms = max_over_ranks(statistics.mean(times), world)
+        res = {"workload": p.name, "value": job_rate(flops, steps, world, t_ms) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": t_ms / steps, "steps": steps, "flops_per_step": flops,
+               "roofline": self.tensor_roofline(flops, kern_ms, "attn_fwd_tc_kernel<128,bf16> (+ prefill_prep_kernel)",
+                                                p.name),
+               "clocks": clocks, "gpu_launches": 2 * steps,
+               "l2": "flushed before every step (512 MiB write)"}
+        hq, hk, hv = p.q.pin_memory(), p.k.pin_memory(), p.v.pin_memory()
+        hcq, hck = p.cu_q.pin_memory(), p.cu_k.pin_memory()
+        ho, hl = torch.empty_like(hq).pin_memory(), torch.empty((p.total_q, p.hq), dtype=torch.float32).pin_memory()
+        dq, dk, dv_ = torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"])
+        dcq, dck = torch.empty_like(d["cu_q"]), torch.empty_like(d["cu_k"])
+
+        def e2e_step():
+            for dst, src in ((dq, hq), (dk, hk), (dv_, hv), (dcq, hcq), (dck, hck)):
+                dst.copy_(src, non_blocking=True)
+            mx.mxfa_attn_varlen_fwd(dq, dk, dv_, dcq, dck, max_q, max_k, causal=True, out=o, lse=lse, ws=ws,
+                                    stream=stream)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        n_e2e = max(5, steps // 3)
+        e2e_times, _ = self.timed(e2e_step, n_e2e, 2)
+        e2e_ms = max_over_ranks(sum(e2e_times), world)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck))
+        res["e2e"] = {"value": job_rate(flops, n_e2e, world, e2e_ms) / 1e12, "unit": "TFLOP/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": ho.numel() * 2 + hl.numel() * 4}
+        res["cpu_baseline"] = cpu_baseline(p, "flops") if self.rank0_cpu else None
+        return res
+
+    # -------- the fp32 single-head problem (us per call)
+    def single_head(self, p, steps):
+        mx, dev, stream, world = self.mx, self.dev, self.stream, self.world
+        S, D = p.meta["Sq"], p.dqk
+        q, k, v = (t.view(1, S, 1, D).to(dev) for t in (p.q, p.k, p.v))
+        o = torch.empty_like(q)
+        lse = torch.empty((1, S, 1), dtype=torch.float32, device=dev)
+        ws = mx.workspace(256, dev)
+
+        def step():
+            mx.mxfa_attn_fwd(q, k, v, causal=False, softmax_scale=p.scale, out=o, lse=lse, ws=ws, stream=stream)
+
+        times, clocks = self.timed(step, steps, self.args.warmup)
+        self.check_status(ws)
+        us = max_over_ranks(statistics.mean(times), world) * 1e3
+        flops = prefill_flops(1, 1, S, D, causal=False)
+        res = {"workload": p.name, "value": us, "unit": "us", "higher_is_better": False, "steps": steps,
+               "tflops": flops / (us / 1e6) / 1e12, "kernel": "attn_fwd_simt_kernel<float> (fp32, CUDA cores)",
+               "bound": "launch latency (4.19 MFLOP)", "clocks": clocks, "gpu_launches": steps,
+               "l2": "flushed before every call (512 MiB write)"}
+        hq, hk, hv = (t.view(1, S, 1, D).pin_memory() for t in (p.q, p.k, p.v))
+        ho, hl = torch.empty_like(hq).pin_memory(), torch.empty((1, S, 1), dtype=torch.float32).pin_memory()
+        dq, dk, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv_.copy_(hv, non_blocking=True)
+            mx.mxfa_attn_fwd(dq, dk, dv_, causal=False, softmax_scale=p.scale, out=o, lse=lse, ws=ws, stream=stream)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_times, _ = self.timed(e2e_step, steps, 2)
+        res["e2e"] = {"value": max_over_ranks(statistics.mean(e2e_times), world) * 1e3, "unit": "us",
+                      "h2d_bytes_per_step": 3 * q.numel() * 4, "d2h_bytes_per_step": o.numel() * 4 + lse.numel() * 4}
+        res["cpu_baseline"] = cpu_baseline_full_us(p) if self.rank0_cpu else None
+        return res
+
+    # -------- decode legs
+    def decode(self, p, steps, kind):
+        mx, dev, stream, world = self.mx, self.dev, self.stream, self.world
+        lib = mx.load()
+        d = workloads.to_device(p, dev)
+        od = torch.empty((p.total_q, p.hq, p.dv), dtype=torch.bfloat16, device=dev)
+        ld = torch.empty((p.total_q, p.hq), dtype=torch.float32, device=dev)
+        max_q, max_k = max(p.seqlens_q()), max(p.seqlens_k())
+        if kind == "fp8":
+            need = lib.mxfa_attn_decode_mla_fp8kv_workspace_size(p.batch, max_q, p.hq, max_k, 0)
+        else:
+            need = lib.mxfa_attn_decode_splitkv_workspace_size(p.batch, max_q, p.hq, p.hkv, p.dv, max_k, 0, 2)
+        wsd = torch.zeros(need + 256, dtype=torch.uint8, device=dev)
+
+        def call(dd, out, lse):
+            if kind == "fp8":
+                mx.mxfa_attn_decode_mla_fp8kv(dd["q"], dd["kv"], p.kv_scale, dd["cu_q"], dd["cu_k"], max_q, max_k,
+                                              softmax_scale=p.scale, out=out, lse=lse, ws=wsd, stream=stream)
+            else:
+                mx.mxfa_attn_decode_splitkv(dd["q"], dd["k"], dd["v"], dd["cu_q"], dd["cu_k"], max_q, max_k,
+                                            softmax_scale=p.scale, out=out, lse=lse, ws=wsd, stream=stream)
+
+        times, clocks = self.timed(lambda: call(d, od, ld), steps, 3, flush=False)
+        self.check_status(wsd)
+        nbytes = decode_bytes(p)
+        ms = max_over_ranks(statistics.mean(times), world)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        key = "decode_gqa" if kind == "gqa" else "decode"
+        res = {"workload": p.name, "value": gbs * world, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
+               "algorithmic_bytes": nbytes, "kv_rows_per_s": p.total_k * world / (ms / 1e3),
+               "l2": "inputs larger than L2", "roofline": self.hbm_roofline(nbytes, ms, key, p.name),
+               "clocks": clocks, "gpu_launches": 3 * steps}
+        # end to end: every input (q, the KV cache, the indptr arrays) copied
+        # from pinned host memory and O, LSE read back, every step
+        hsrc = {"q": p.q, "cu_q": p.cu_q, "cu_k": p.cu_k}
+        if p.mla:
+            hsrc["kv"] = p.kv
+        else:
+            hsrc["k"], hsrc["v"] = p.k, p.v
+        hsrc = {n: t.contiguous().pin_memory() for n, t in hsrc.items()}
+        dsrc = {n: torch.empty_like(t, device=dev) for n, t in hsrc.items()}
+        if p.mla:
+            dsrc["k"] = dsrc["kv"].view(-1, 1, p.dqk)
+            dsrc["v"] = dsrc["kv"][:, :p.dv].view(-1, 1, p.dv)
+        ho, hl = torch.empty(od.shape, dtype=od.dtype).pin_memory(), torch.empty(ld.shape).pin_memory()
+
+        def e2e_step():
+            for n, t in hsrc.items():
+                dsrc[n].copy_(t, non_blocking=True)
+            call(dsrc, od, ld)
+            ho.copy_(od, non_blocking=True)
+            hl.copy_(ld, non_blocking=True)
+
+        n_e2e = 5
+        e2e_times, _ = self.timed(e2e_step, n_e2e, 2, flush=False)
+        e2e_ms = max_over_ranks(statistics.mean(e2e_times), world)
+        res["e2e"] = {"value": nbytes * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+                      "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hsrc.values()),
+                      "d2h_bytes_per_step": ho.numel() * 2 + hl.numel() * 4,
+                      "note": "the KV cache crosses PCIe every step here; in serving it stays resident"}
+        if kind == "fp8":
+            # the oracle dequantises the whole cache to fp64 (4.8 GB) per call,
+            # which the host run does not afford; the bf16 decode line carries
+            # the oracle's rate on the same shape
+            res["cpu_baseline"] = None
+        else:
+            res["cpu_baseline"] = cpu_baseline(p, "bytes", full_units=nbytes) if self.rank0_cpu else None
+        del d, dsrc
+        return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="mxfa", choices=["mxfa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--only", default=None,
+                    choices=["headline", "batched_causal", "varlen_gqa", "single_head_fp32", "decode", "gqa", "fp8"],
+                    help="time one workload only (used for profiling captures; no JSON contract line)")
     ap.add_argument("--decode-batch", type=int, default=128,
-                    help="sequences of the MLA decode workload (128 = the full workload; smaller for captures)")
-    ap.add_argument("--only", choices=["prefill", "decode", "gqa", "fp8"], default=None,
-                    help="time one workload only (used for profiling captures)")
+                    help="sequences of the MLA decode workloads (128 = the full workload; smaller for captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -280,173 +598,49 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     import tiled_attention_21_b200 as mx
     mx.load()
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from runners import to_dev
-
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
-    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    bn = Bench(args, world, local, dev, stream)
+    want = (lambda name: args.only in (None, name))
+    out = {}
 
-    def flush():
-        flush_buf.zero_()
-
-    pk, pk_kind = peaks()
-
-    # ---------------- prefill (the step)
-    B, H, S, D = PREFILL_CFG["B"], PREFILL_CFG["H"], PREFILL_CFG["S"], PREFILL_CFG["D"]
-    p = workloads.cfg_batched_causal()
-    q = p.q.view(B, S, H, D).to(dev)
-    k = p.k.view(B, S, H, D).to(dev)
-    v = p.v.view(B, S, H, D).to(dev)
-    o = torch.empty_like(q)
-    lse = torch.empty((B, S, H), dtype=torch.float32, device=dev)
-    ws = mx.workspace(256, dev)
-
-    def step():
-        mx.mxfa_attn_fwd(q, k, v, causal=True, out=o, lse=lse, ws=ws, stream=stream)
-
-    flops = prefill_flops(B, H, S, D)
-    if args.only in ("decode", "gqa", "fp8"):
-        args.steps = 0
-    with ClockSampler(local) as clk:
-        times = time_steps(step, args.steps, args.warmup, flush, stream, world)
-    st, site = mx.read_device_status(ws)
-    if st != 0:
-        raise RuntimeError(f"device status {st} at site 0x{site:x}")
-    t_ms = max_over_ranks(sum(times), world) if times else float("nan")
-    ms_per_step = t_ms / max(1, args.steps)
-    value = job_rate(flops, args.steps, world, t_ms) / 1e12 if times else float("nan")
-    kern_ms = statistics.mean(times) if times else float("nan")  # one kernel launch per step
-    achieved = flops / (kern_ms / 1e3) / 1e12
-    traffic = recorded_traffic("attn_fwd_tc_kernel", "batched_causal_b4_h16_s2048_d128_bf16")
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_tflops"], "traffic": traffic, "kernel": "attn_fwd_tc_kernel<128,bf16>",
-                "peak_kind": f"{pk_kind} burst dense bf16 (cuBLAS)"}
-
-    # ---------------- e2e through the public API with host buffers
-    hq = p.q.view(B, S, H, D).pin_memory()
-    hk = p.k.view(B, S, H, D).pin_memory()
-    hv = p.v.view(B, S, H, D).pin_memory()
-    ho = torch.empty((B, S, H, D), dtype=torch.bfloat16).pin_memory()
-    hl = torch.empty((B, S, H), dtype=torch.float32).pin_memory()
-    dq, dk, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv_.copy_(hv, non_blocking=True)
-        mx.mxfa_attn_fwd(dq, dk, dv_, causal=True, out=o, lse=lse, ws=ws, stream=stream)
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
-
-    e2e_times = time_steps(e2e_step, max(5, args.steps // 3), 3, flush, stream, world) if args.only is None else [1.0]
-    e2e_ms = max_over_ranks(sum(e2e_times), world)
-    e2e_val = flops * len(e2e_times) * world / (e2e_ms / 1e3) / 1e12
-    h2d = 3 * q.numel() * 2
-    d2h = o.numel() * 2 + lse.numel() * 4
-
-    # ---------------- decode (secondary measurement)
-    decode = None
-    if not args.no_decode and args.only in (None, "decode"):
+    if want("headline"):
+        out["headline"] = bn.batched_prefill(headline_problem(), args.steps)
+    if want("batched_causal"):
+        out["batched_causal"] = bn.batched_prefill(workloads.cfg_batched_causal(), args.steps)
+    if want("varlen_gqa"):
+        out["varlen_gqa"] = bn.varlen_prefill(workloads.cfg_varlen_gqa(), args.steps)
+    if want("single_head_fp32"):
+        out["single_head_fp32"] = bn.single_head(workloads.cfg_single_head_fp32(), args.steps)
+    dsteps = max(5, args.steps // 2)
+    if want("decode"):
         pdc = (workloads.cfg_mla_decode() if args.decode_batch == 128 else
-               workloads.mla_decode(3, args.decode_batch, 4, 8192, name=f"mla_decode_b{args.decode_batch}_q4_h16_kv8192_bf16"))
-        dd = to_dev(pdc, dev)
-        od = torch.empty((pdc.total_q, pdc.hq, pdc.dv), dtype=torch.bfloat16, device=dev)
-        ld = torch.empty((pdc.total_q, pdc.hq), dtype=torch.float32, device=dev)
-        need = mx.load().mxfa_attn_decode_splitkv_workspace_size(pdc.batch, 4, pdc.hq, 1, pdc.dv, 8192, 0, 2)
-        wsd = torch.zeros(need + 256, dtype=torch.uint8, device=dev)
-
-        def dstep():
-            mx.mxfa_attn_decode_splitkv(dd["q"], dd["k"], dd["v"], dd["cu_q"], dd["cu_k"], 4, 8192,
-                                        softmax_scale=pdc.scale, out=od, lse=ld, ws=wsd, stream=stream)
-
-        dsteps = max(5, args.steps // 3)
-        dtimes = time_steps(dstep, dsteps, 3, lambda: None, stream, world)  # KV (1.2 GB) >> L2
-        dbytes = decode_bytes(pdc)
-        dms = max_over_ranks(statistics.mean(dtimes), world)
-        dgbs = dbytes / (dms / 1e3) / 1e9
-        decode = {"workload": pdc.name, "value": dgbs * world, "unit": "GB/s", "ms_per_step": dms,
-                  "algorithmic_bytes": dbytes, "l2": "inputs (1.2 GB KV) larger than L2",
-                  "roofline": {"bound": "hbm", "achieved": dgbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                               "frac": dgbs / pk["hbm_gbs"],
-                               "traffic": recorded_traffic("decode", "mla_decode_b128_q4_h16_kv8192_bf16"),
-                               "peak_kind": f"{pk_kind} HBM copy"}}
-
-    # ---------------- grouped-query decode (next scope row; secondary measurement)
-    decode_gqa = None
-    if not args.no_decode and args.only in (None, "gqa"):
-        pg = workloads.cfg_gqa_decode()
-        dg = to_dev(pg, dev)
-        og = torch.empty((pg.total_q, pg.hq, pg.dv), dtype=torch.bfloat16, device=dev)
-        lg = torch.empty((pg.total_q, pg.hq), dtype=torch.float32, device=dev)
-        kvl = pg.total_k // pg.batch
-        need = mx.load().mxfa_attn_decode_splitkv_workspace_size(pg.batch, 1, pg.hq, pg.hkv, pg.dv, kvl, 0, 2)
-        wsg = torch.zeros(need + 256, dtype=torch.uint8, device=dev)
-
-        def gstep():
-            mx.mxfa_attn_decode_splitkv(dg["q"], dg["k"], dg["v"], dg["cu_q"], dg["cu_k"], 1, kvl,
-                                        softmax_scale=pg.scale, out=og, lse=lg, ws=wsg, stream=stream)
-
-        gtimes = time_steps(gstep, max(5, args.steps // 3), 3, lambda: None, stream, world)  # KV 1.07 GB >> L2
-        gbytes = decode_bytes(pg)
-        gms = max_over_ranks(statistics.mean(gtimes), world)
-        ggbs = gbytes / (gms / 1e3) / 1e9
-        decode_gqa = {"workload": pg.name, "value": ggbs * world, "unit": "GB/s", "ms_per_step": gms,
-                      "algorithmic_bytes": gbytes, "l2": "inputs (1.07 GB K+V) larger than L2",
-                      "roofline": {"bound": "hbm", "achieved": ggbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                   "frac": ggbs / pk["hbm_gbs"],
-                                   "traffic": recorded_traffic("decode_gqa", pg.name),
-                                   "peak_kind": f"{pk_kind} HBM copy"}}
-
-    # ---------------- MLA decode over an E4M3 cache (next scope row; secondary measurement)
-    decode_fp8 = None
-    if not args.no_decode and args.only in (None, "fp8"):
-        pf = workloads.cfg_mla_decode_fp8()
-        df = to_dev(pf, dev)
-        of = torch.empty((pf.total_q, pf.hq, pf.dv), dtype=torch.bfloat16, device=dev)
-        lf = torch.empty((pf.total_q, pf.hq), dtype=torch.float32, device=dev)
-        need = mx.load().mxfa_attn_decode_mla_fp8kv_workspace_size(pf.batch, 4, pf.hq, 8192, 0)
-        wsf = torch.zeros(need + 256, dtype=torch.uint8, device=dev)
-
-        def fstep():
-            mx.mxfa_attn_decode_mla_fp8kv(df["q"], df["kv"], pf.kv_scale, df["cu_q"], df["cu_k"], 4, 8192,
-                                          softmax_scale=pf.scale, out=of, lse=lf, ws=wsf, stream=stream)
-
-        ftimes = time_steps(fstep, max(5, args.steps // 3), 3, lambda: None, stream, world)  # 604 MB codes >> L2
-        fbytes = decode_bytes(pf)
-        fms = max_over_ranks(statistics.mean(ftimes), world)
-        fgbs = fbytes / (fms / 1e3) / 1e9
-        fflops = 2.0 * pf.total_q * pf.hq * (pf.total_k // pf.batch) * (pf.dqk + pf.dv)
-        decode_fp8 = {"workload": pf.name, "value": fgbs * world, "unit": "GB/s", "ms_per_step": fms,
-                      "algorithmic_bytes": fbytes, "l2": "inputs (604 MB of codes) larger than L2",
-                      "kv_rows_per_s": pf.total_k * world / (fms / 1e3),
-                      "mma_tflops": fflops / (fms / 1e3) / 1e12,
-                      "limit": "not HBM: the same M = 64 bf16 MMAs per KV row as the bf16 cache, plus the "
-                               "shared-memory traffic of widening the codes; compare kv_rows_per_s with decode's",
-                      "roofline": {"bound": "hbm", "achieved": fgbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                                   "frac": fgbs / pk["hbm_gbs"],
-                                   "traffic": recorded_traffic("decode", pf.name),
-                                   "peak_kind": f"{pk_kind} HBM copy"}}
-        if decode is not None:
-            decode["kv_rows_per_s"] = pdc.total_k * world / (decode["ms_per_step"] / 1e3)
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only is None:
-        cpu = cpu_baseline_prefill()
+               workloads.mla_decode(3, args.decode_batch, 4, 8192,
+                                    name=f"mla_decode_b{args.decode_batch}_q4_h16_kv8192_bf16"))
+        out["decode"] = bn.decode(pdc, dsteps, "mla")
+    if want("gqa"):
+        out["decode_gqa"] = bn.decode(workloads.cfg_gqa_decode(), dsteps, "gqa")
+    if want("fp8"):
+        pf = (workloads.cfg_mla_decode_fp8() if args.decode_batch == 128 else
+              workloads.mla_decode_fp8(3, args.decode_batch, 4, 8192,
+                                       name=f"mla_decode_b{args.decode_batch}_q4_h16_kv8192_fp8kv"))
+        out["decode_fp8"] = bn.decode(pf, dsteps, "fp8")
+        out["decode_fp8"]["mma_tflops"] = (2.0 * pf.total_q * pf.hq * (pf.total_k // pf.batch) * (pf.dqk + pf.dv)
+                                           / (out["decode_fp8"]["ms_per_step"] / 1e3) / 1e12)
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": p.name, "B": B, "H": H, "seq_len": S, "head_dim": D, "causal": True,
-                           "flops_per_step": flops, "l2": "flushed before every step (512 MiB write)",
-                           "parallelism": f"replicas x{world}"},
-                "roofline": roofline, "cpu_baseline": cpu,
-                "e2e": None if args.only else {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                                               "d2h_bytes_per_step": d2h},
-                "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
-                "decode_gqa": decode_gqa, "decode_fp8": decode_fp8}
-        print(json.dumps(line), flush=True)
+        if args.only is not None:
+            print(json.dumps(out), flush=True)
+        else:
+            h = out.pop("headline")
+            line = {"metric": METRIC, "value": h["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                    "warmup": args.warmup, "ms_per_step": h["ms_per_step"], "higher_is_better": True,
+                    "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                    "config": headline_config_of(h["workload"], h["flops_per_step"], world),
+                    "roofline": h["roofline"], "cpu_baseline": h["cpu_baseline"], "e2e": h["e2e"],
+                    "gpu_launches": h["gpu_launches"], "clocks": h["clocks"]}
+            line.update(out)
+            print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -131,12 +131,28 @@ mxfa_status_t mxfa_attn_varlen_fwd(const void *q, const void *k, const void *v, 
  *     streams without ordering, or several host threads) race and must not
  *     be issued; order them on one stream.
  *   - No device memory is allocated or freed.
+ *   - A rejected call (any check of mxfa_attn_varlen_fwd, or the size
+ *     limit) writes nothing; an accepted one first clears the status word
+ *     at the head of the array, so read it (mxfa_read_noalloc_status) after
+ *     a call and before the next one.
  */
 mxfa_status_t mxfa_attn_varlen_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
                                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
                                            int batch, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
                                            int Hq, int Hkv, int D, mxfa_dtype_t dtype,
                                            float softmax_scale, int causal, void *stream);
+
+/*
+ * Device-side status of the last mxfa_attn_varlen_fwd_noalloc call on the
+ * current device: what mxfa_read_device_status returns for a caller
+ * workspace (MXFA_OK; MXFA_ERR_TIMEOUT when a bounded wait gave up;
+ * MXFA_ERR_INVALID_ARG when a sequence was longer than max_seqlen_q, so
+ * part of O was not written), read from the library's scratch array.
+ * Synchronises `stream`, clears the word when it is set, and sets
+ * mxfa_device_status_detail() to the site code.  No pages have a
+ * counterpart.
+ */
+mxfa_status_t mxfa_read_noalloc_status(void *stream);
 
 /*
  * Split-KV decode (few queries per sequence, long KV), with the partial
@@ -257,14 +273,36 @@ const char *mxfa_last_error(void);
  * Synchronises `stream`, reads the status word the last call wrote into
  * `workspace` and returns it (MXFA_OK, or MXFA_ERR_TIMEOUT when a bounded
  * device wait gave up; the kernel then skipped its remaining work and left
- * the outputs incomplete).  mxfa_device_status_detail() returns the site
- * code of that wait from the same read.
+ * the outputs incomplete), and clears it when it is set.
+ * mxfa_device_status_detail() returns the site code from the same read:
+ * for a timeout the wait that ran out; for MXFA_ERR_INVALID_ARG 0x201 (a
+ * varlen sequence longer than max_seqlen_q: its blocks beyond the schedule
+ * were not computed), 0x401 (decode pieces beyond the workspace schedule)
+ * or 0x402 (a KV-cache length beyond the cache's capacity: attention ran
+ * over the first page_size keys of a dense entry, or max_blocks_per_seq
+ * pages of a paged one).
  */
 mxfa_status_t mxfa_read_device_status(const void *workspace, void *stream);
 uint32_t mxfa_device_status_detail(void);
 
 /* Library version, (major << 16) | (minor << 8) | patch. */
 uint32_t mxfa_version(void);
+
+/*
+ * Testing hooks (for the library's own tests; the pages have no
+ * counterpart).  Process-wide settings read by every later call:
+ *   wait_budget_ns: budget of every bounded device-side wait of later
+ *     launches, in nanoseconds (0 restores the default of 2 s).  A wait that
+ *     runs out records MXFA_ERR_TIMEOUT and its site code in the workspace
+ *     status word and the kernel returns without finishing its work.
+ *   keep_merge_counters: non-zero makes the one-launch decode schedule (see
+ *     mxfa_attn_decode_splitkv) skip its memset of the per-sequence merge
+ *     counters and use the values the caller left in the workspace; a
+ *     counter that cannot reach its sequence's piece count makes the merge
+ *     wait run out (its site code is 0x309).
+ * Production code does not call this.
+ */
+void mxfa_test_hooks(uint64_t wait_budget_ns, int keep_merge_counters);
 
 #ifdef __cplusplus
 }

@@ -26,18 +26,32 @@ def half_ulp(x: torch.Tensor, dtype) -> torch.Tensor:
     return 0.5 * torch.pow(2.0, e - (MANT[dtype] - 1))
 
 
+# Figures of the last compare() call: the max-abs error against the oracle,
+# against the oracle rounded to the output format (what a correctly rounded
+# kernel would store), and the number of elements whose exact value has
+# magnitude >= 4 (where the output rounding alone can exceed 1e-2).
+LAST: dict = {}
+
+
 def compare(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what="", lse_tol=None):
     """o_gpu / lse_gpu: device or host tensors shaped like o_ref / lse_ref (fp64).
-    lse_tol overrides the LSE bound (a float, or a tensor per row)."""
+    lse_tol overrides the LSE bound (a float, or a tensor per row).  Every
+    failure message carries the figures of ``LAST``."""
     o = o_gpu.detach().double().cpu()
     assert torch.isfinite(o).all(), f"{what}: non-finite output"
     err = (o - o_ref).abs()
     tol = TOL_O[dtype]
     small = o_ref.abs() < 4.0
+    LAST.clear()
+    LAST.update(max_abs=err.max().item() if err.numel() else 0.0,
+                max_abs_vs_rounded=(o - o_ref.to(dtype).double()).abs().max().item() if err.numel() else 0.0,
+                n_big=int((~small).sum()))
+    figs = (f"max|dO| {LAST['max_abs']:.3e}, vs oracle rounded to {dtype}: {LAST['max_abs_vs_rounded']:.3e}, "
+            f"{LAST['n_big']} elements with |O| >= 4")
     assert err[small].numel() == 0 or err[small].max().item() <= tol, \
-        f"{what}: max |dO| = {err[small].max().item():.3e} > {tol}"
+        f"{what}: max |dO| = {err[small].max().item():.3e} > {tol} ({figs})"
     big_tol = tol + half_ulp(o_ref, dtype)
-    assert bool((err <= big_tol).all()), f"{what}: |dO| beyond tolerance + output rounding"
+    assert bool((err <= big_tol).all()), f"{what}: |dO| beyond tolerance + output rounding ({figs})"
     if lse_gpu is not None:
         l = lse_gpu.detach().double().cpu()
         fin = torch.isfinite(lse_ref)

@@ -1,17 +1,6 @@
 """Run a workloads.Problem through the library's public entry points (test/bench helper)."""
-import torch
-
 import tiled_attention_21_b200 as mx
-
-
-def to_dev(p, device="cuda"):
-    d = {"q": p.q.to(device), "k": p.k.to(device), "v": p.v.to(device),
-         "cu_q": p.cu_q.to(device), "cu_k": p.cu_k.to(device)}
-    if p.mla:
-        d["kv"] = p.kv.to(device)
-        d["k"] = d["kv"].view(-1, 1, p.dqk)
-        d["v"] = d["kv"][:, :p.dv].view(-1, 1, p.dv)
-    return d
+from workloads import to_device as to_dev  # noqa: F401  (re-exported for the tests)
 
 
 def run(p, d, entry=None, num_splits=0, stream=None, out=None, lse=None):

@@ -94,3 +94,22 @@ def test_append_past_capacity_is_reported():
     st, site = mx.read_device_status(ws)
     assert st == mx.MXFA_ERR_INVALID_ARG and site == 0x501
     assert torch.equal(kc, kc0)  # nothing written
+
+
+def test_dense_length_past_capacity_is_reported():
+    """A dense cache entry holds page_size (= the cache length) keys; a
+    cache_seqlens value beyond it is cut there and reported (site 0x402), so
+    no key of the next entry is read."""
+    import tiled_attention_21_b200 as mx
+    dev = torch.device("cuda")
+    w = workloads.kvcache(47, batch=2, Sq=1, Snew=0, seqlens=[64, 30], cache_len=64)
+    kc, vc = w["k_cache"].to(dev), w["v_cache"].to(dev)
+    sl = torch.tensor([100, 30], dtype=torch.int32, device=dev)
+    ws = mx.workspace(1 << 20, dev)
+    o, lse = mx.mxfa_attn_decode_kvcache(w["q"].to(dev), kc, vc, sl, ws=ws)
+    st, site = mx.read_device_status(ws)
+    assert (st, site) == (mx.MXFA_ERR_INVALID_ARG, 0x402)
+    p = w["problem"]  # the 64 cached keys of entry 0, 30 of entry 1
+    ro, rl = oracle.problem(p)
+    B, Sq, Hq, D = w["q"].shape
+    compare(o.reshape(B * Sq, Hq, D), lse.reshape(B * Sq, Hq), ro, rl, p.q.dtype, "dense past capacity")

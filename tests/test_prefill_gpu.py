@@ -179,3 +179,22 @@ def test_full_size_varlen_gqa_sampled():
 
 def test_full_size_long_context_sampled():
     _sampled(workloads.cfg_long_causal(), 0, 103)
+
+
+def test_varlen_max_seqlen_below_a_length_is_reported():
+    """max_seqlen_q sizes the varlen schedule; a sequence longer than it
+    leaves 256-row blocks unscheduled, which the schedule kernel reports as
+    MXFA_ERR_INVALID_ARG at site 0x201 (strict mode off, so the host does not
+    read cu_seqlens)."""
+    import tiled_attention_21_b200 as mx
+    p = workloads.varlen(19, [1000, 10], [1000, 10], 4, 4, 128, "bf16", True)
+    d = to_dev(p)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    mx.mxfa_attn_varlen_fwd(d["q"], d["k"], d["v"], d["cu_q"], d["cu_k"], 300, 1000, causal=True, ws=ws)
+    st, site = mx.read_device_status(ws)
+    assert (st, site) == (mx.MXFA_ERR_INVALID_ARG, 0x201)
+    # the status was cleared by the read; a call with the true maximum is clean
+    o, l = mx.mxfa_attn_varlen_fwd(d["q"], d["k"], d["v"], d["cu_q"], d["cu_k"], 1000, 1000, causal=True, ws=ws)
+    assert mx.read_device_status(ws)[0] == mx.MXFA_OK
+    ro, rl = oracle.problem(p)
+    compare(o, l, ro, rl, p.q.dtype, p.name)

@@ -74,6 +74,12 @@ def load():
             lib.mxfa_device_status_detail.restype = ctypes.c_uint32
             lib.mxfa_version.argtypes = []
             lib.mxfa_version.restype = ctypes.c_uint32
+            lib.mxfa_attn_varlen_fwd_noalloc.argtypes = [vp] * 7 + [i32] * 9 + [f32, i32, vp]
+            lib.mxfa_attn_varlen_fwd_noalloc.restype = i32
+            lib.mxfa_read_noalloc_status.argtypes = [vp]
+            lib.mxfa_read_noalloc_status.restype = i32
+            lib.mxfa_test_hooks.argtypes = [ctypes.c_uint64, i32]
+            lib.mxfa_test_hooks.restype = None
             _lib = lib
     return _lib
 
@@ -121,6 +127,14 @@ def read_device_status(ws: torch.Tensor | None = None, device=None) -> tuple[int
         ws = workspace(256, device or torch.device("cuda"))
     p, _ = _ws_view(ws)
     st = lib.mxfa_read_device_status(ctypes.c_void_p(p), _stream(None))
+    return st, lib.mxfa_device_status_detail()
+
+
+def read_noalloc_status(stream=None) -> tuple[int, int]:
+    """(status, site) of the no-allocation varlen entry point's last call on
+    the current device (its scratch array's status word); clears it."""
+    lib = load()
+    st = lib.mxfa_read_noalloc_status(_stream(stream))
     return st, lib.mxfa_device_status_detail()
 
 
@@ -283,5 +297,6 @@ def mxfa_attn_decode_kvcache(q, k_cache, v_cache, cache_seqlens, k_new=None, v_n
     return out, lse
 
 
-__all__ = ["load", "mxfa_attn_fwd", "mxfa_attn_varlen_fwd", "mxfa_attn_decode_splitkv", "mxfa_attn_decode_kvcache",
-           "read_device_status", "workspace", "MxfaError", "LIB_PATH"]
+__all__ = ["load", "mxfa_attn_fwd", "mxfa_attn_varlen_fwd", "mxfa_attn_decode_splitkv", "mxfa_attn_decode_mla_fp8kv",
+           "mxfa_attn_decode_kvcache", "read_device_status", "read_noalloc_status", "workspace", "MxfaError",
+           "LIB_PATH"]

@@ -23,7 +23,8 @@ static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 constexpr uint32_t kStatusTimeout = 5;  // == MXFA_ERR_TIMEOUT
 
-// Wait budget of every device-side spin, in nanoseconds of %globaltimer.
+// Default wait budget of every device-side spin, in nanoseconds of
+// %globaltimer; each launch carries its budget in AttnParams::wait_ns.
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -53,6 +54,7 @@ struct AttnParams {
   int causal;
   WsHeader *hdr;
   const int2 *pairs;          // varlen schedule: sorted (sequence, 256-row block) pairs
+  uint64_t wait_ns;           // budget of every bounded device-side wait (kWaitBudgetNs unless a test shortens it)
 };
 
 struct SeqRange {

@@ -128,7 +128,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
         const int len = dc_klen(p, s, b);
         for (int j = sd.y; ok && j < sd.z; ++j, ++tc) {
           const int x = tc % Cfg::kRingTiles;
-          if (!wait_bar(b_te(x), ((tc / Cfg::kRingTiles) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty)) {
+          if (!wait_bar(b_te(x), ((tc / Cfg::kRingTiles) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -155,7 +155,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
       for (int x = 0; x < Cfg::kRingTiles; ++x) {
         const uint32_t uses = tc / Cfg::kRingTiles + ((uint32_t)x < tc % Cfg::kRingTiles ? 1u : 0u);
         if (uses == 0) continue;
-        while (!mbar_test(b_tf(x), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        while (!mbar_test(b_tf(x), (uses - 1) & 1) && global_ns() - t0 < p.wait_ns) {
         }
       }
     }
@@ -165,7 +165,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     // lane issues each tcgen05 operation; the warp gives up a wait together.
     const bool leader = elect_one();
     auto wait_warp = [&](uint32_t bar, uint32_t parity, uint32_t site) {
-      return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, hdr, site));
+      return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, hdr, site, p.wait_ns));
     };
     constexpr uint32_t idesc_s = make_idesc_f16(BF16, kDcRows, kGqKeys, false, false);
     constexpr uint32_t idesc_o = make_idesc_f16(BF16, kDcRows, D, false, true);
@@ -234,7 +234,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     }
     if (leader) mma_commit(smem_u32(&ctrl->drain));
     const uint64_t t0 = global_ns();
-    while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < kWaitBudgetNs) {
+    while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < p.wait_ns) {
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax / epilogue
@@ -278,7 +278,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
       const int nv = valid ? visible_keys(r / G, sq, sk, p.causal) : 0;
       float m_used = -INFINITY, l = 0.f;
       for (int j = sd.y; j < sd.z; ++j, ++g) {
-        const bool got = wait_bar(b_sf, g & 1, abort_flag, hdr, kDSiteSFull);
+        const bool got = wait_bar(b_sf, g & 1, abort_flag, hdr, kDSiteSFull, p.wait_ns);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
@@ -337,7 +337,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
         l = l * alpha + rs;
         // P (single buffer) and O may be touched only once the previous P.V is done.
         if (g > 0) {
-          const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone);
+          const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got_o)) {
             ok = false;
@@ -378,7 +378,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
       // ---------------- epilogue of this piece
       l += __shfl_xor_sync(0xffffffffu, l, 16);
       if (sd.z > sd.y) {
-        const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone);
+        const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got_o)) break;
         tc_fence_after();

@@ -232,8 +232,18 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     int n = 0;
     if (b < B) {
       const int e = b / s.heads;  // batch entry of sequence b
-      const int len = p.cu_k ? p.cu_k[e + 1] - p.cu_k[e] : s.cache_seqlens[e] + s.add;
-      if (!p.cu_k && b % s.heads == 0) s.kv_len[e] = len;
+      int len = p.cu_k ? p.cu_k[e + 1] - p.cu_k[e] : s.cache_seqlens[e] + s.add;
+      if (!p.cu_k) {
+        // A cache entry holds at most page_size keys (dense) or max_blocks
+        // pages (paged); positions beyond would read another entry's rows or
+        // no page at all, so the length is cut there and the call reports it.
+        const int64_t cap = s.block_table ? (int64_t)s.max_blocks * s.page_size : (int64_t)s.page_size;
+        if (len > cap) {
+          if (b % s.heads == 0) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x402);
+          len = (int)cap;
+        }
+        if (b % s.heads == 0) s.kv_len[e] = len;
+      }
       n = (len + s.keys - 1) / s.keys;
       if (dc_q(p, e).y <= 0) n = 0;  // no queries: nothing to compute
       s.n_tiles[b] = n;
@@ -379,7 +389,7 @@ __device__ void dc_merge_pieces(const AttnParams &p, const DecodeSched &s, int v
     const uint64_t t0 = global_ns();
     int good = 1;
     while (*reinterpret_cast<volatile int *>(s.sync + v) < k) {
-      if (global_ns() - t0 > kWaitBudgetNs) {
+      if (global_ns() - t0 > p.wait_ns) {
         report_error(p.hdr, kStatusTimeout, kDSiteMerge);
         good = 0;
         break;
@@ -606,7 +616,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         }
         for (int j = sd.y; ok && j < sd.z; ++j, ++tc) {
           const int x = tc % RT;
-          if (!wait_bar(b_te(x), ((tc / RT) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty)) {
+          if (!wait_bar(b_te(x), ((tc / RT) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -633,9 +643,9 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       for (int x = 0; x < RT; ++x) {
         const uint32_t uses = tc / RT + ((uint32_t)x < tc % RT ? 1u : 0u);
         if (uses == 0) continue;
-        while (!mbar_test(FP8 ? b_gf(x) : b_tf(x), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        while (!mbar_test(FP8 ? b_gf(x) : b_tf(x), (uses - 1) & 1) && global_ns() - t0 < p.wait_ns) {
         }
-        while (FP8 && !mbar_test(b_gr(x), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        while (FP8 && !mbar_test(b_gr(x), (uses - 1) & 1) && global_ns() - t0 < p.wait_ns) {
         }
       }
     }
@@ -646,7 +656,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     // the warp gives up a wait together if any lane gave up.
     const bool leader = elect_one();
     auto wait_warp = [&](uint32_t bar, uint32_t parity, volatile int *ab, WsHeader *h, uint32_t site) {
-      return __all_sync(0xffffffffu, wait_bar(bar, parity, ab, h, site));
+      return __all_sync(0xffffffffu, wait_bar(bar, parity, ab, h, site, p.wait_ns));
     };
     {
       constexpr uint32_t idesc_s = make_idesc_f16(BF16, kDcRows, kDcKeys, false, false);
@@ -736,7 +746,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       }
       if (leader) mma_commit(smem_u32(&ctrl->drain));
       const uint64_t t0 = global_ns();
-      while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < kWaitBudgetNs) {
+      while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < p.wait_ns) {
       }
     }
   } else if (FP8 && (warp >= 8 || warp == 2 || warp == 3)) {
@@ -780,7 +790,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       const int4 sd = dc_seg(p, s, sg);
       for (int j = sd.y; j < sd.z; ++j, ++tc) {
         const int y = tc % RT;
-        if (!agree(wait_bar(b_gf(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull))) {
+        if (!agree(wait_bar(b_gf(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -793,7 +803,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         mbar_arrive(b_lf(y));  // S may start on chunks 0-2
         // chunks 3-8 (from chunk 4 on) overwrite codes: every thread reads
         // its groups (and has read its chunk 0-2 groups) before any write
-        if (!agree(wait_bar(b_gr(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull))) {
+        if (!agree(wait_bar(b_gr(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -864,7 +874,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       const int nv = valid ? visible_keys(r / p.hq, sq, sk, p.causal) : 0;
       float m_used = -INFINITY, l = 0.f;
       for (int j = sd.y; j < sd.z; ++j, ++g) {
-        const bool got = wait_bar(b_sf, g & 1, abort_flag, hdr, kDSiteSFull);
+        const bool got = wait_bar(b_sf, g & 1, abort_flag, hdr, kDSiteSFull, p.wait_ns);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
@@ -915,7 +925,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         l = l * alpha + rs;
         // P (single buffer) and O may be touched only once the previous P.V is done.
         if (g > 0) {
-          const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone);
+          const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got_o)) {
             ok = false;
@@ -951,7 +961,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       // ---------------- epilogue of this piece
       l += __shfl_xor_sync(0xffffffffu, l, 16);
       if (sd.z > sd.y) {
-        const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone);
+        const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got_o)) break;
         tc_fence_after();

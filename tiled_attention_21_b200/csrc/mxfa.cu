@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -237,6 +238,13 @@ mxfa_status_t strict_check_cu(const int32_t *cu, int batch, int total, int max_l
 
 float resolve_scale(float s, int dqk) { return std::isnan(s) ? 1.0f / std::sqrt((float)dqk) : s; }
 
+// Testing hooks (mxfa_test_hooks): the budget of every bounded device wait
+// of later launches, and whether the one-launch decode leaves its merge
+// counters as the caller prepared them in the workspace instead of zeroing
+// them.  Process-wide; the defaults are the production behaviour.
+std::atomic<uint64_t> g_wait_ns{kWaitBudgetNs};
+std::atomic<int> g_keep_merge_counters{0};
+
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- launchers
@@ -434,7 +442,8 @@ mxfa_status_t launch_decode_gqa_t(AttnParams &p, const DecodeSched &s, mxfa_dtyp
     DecodeSched sa = s;
     const int t_min = max_tiles > 16 ? 4 : 2;  // tiles per piece at least (merge cost vs chain length)
     sa.arith_k = std::max(1, std::min(s.grid / n_seq, (max_tiles + t_min - 1) / t_min));
-    if (sa.arith_k > 1) MXFA_CUDA(cudaMemsetAsync(sa.sync, 0, sizeof(int) * (size_t)n_seq, st));
+    if (sa.arith_k > 1 && !g_keep_merge_counters.load())
+      MXFA_CUDA(cudaMemsetAsync(sa.sync, 0, sizeof(int) * (size_t)n_seq, st));
     MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(k), GqaCfg<D>::kSmemBytes));
     void *args[] = {&p, &sa, &mk, &mv};
     MXFA_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(k), dim3(n_seq * sa.arith_k),
@@ -493,7 +502,8 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
     DecodeSched sa = s;
     const int t_min = max_tiles > 32 ? 4 : 2;  // tiles per piece at least (merge cost vs chain length)
     sa.arith_k = std::max(1, std::min(s.grid / p.batch, (max_tiles + t_min - 1) / t_min));
-    if (sa.arith_k > 1) MXFA_CUDA(cudaMemsetAsync(sa.sync, 0, sizeof(int) * (size_t)p.batch, st));
+    if (sa.arith_k > 1 && !g_keep_merge_counters.load())
+      MXFA_CUDA(cudaMemsetAsync(sa.sync, 0, sizeof(int) * (size_t)p.batch, st));
     void *args[] = {&p, &sa, &mq, &mkv};
     MXFA_CUDA(cudaLaunchCooperativeKernel(k, dim3(p.batch * sa.arith_k), dim3(threads), args, kDcSmemBytes, st));
     return MXFA_OK;
@@ -517,6 +527,71 @@ mxfa_status_t check_heads(int Hq, int Hkv) {
   return MXFA_OK;
 }
 
+// ---------------------------------------------------------------- varlen forward
+// The arguments of mxfa_attn_varlen_fwd, checked and launched in steps so
+// that the entry point with a caller workspace and the one with the
+// library's scratch array run the same checks before either touches device
+// memory.
+struct VarlenArgs {
+  const void *q, *k, *v;
+  void *o;
+  float *lse;
+  const int32_t *cu_q, *cu_k;
+  int batch, total_q, total_k, max_q, max_k, Hq, Hkv, D;
+  mxfa_dtype_t dtype;
+  float scale;
+  int causal;
+};
+
+// Host-side checks; *noop is set for an empty problem (nothing to launch).
+mxfa_status_t varlen_check(const VarlenArgs &a, bool *noop) {
+  *noop = false;
+  if (!dtype_ok(a.dtype)) return fail(MXFA_ERR_INVALID_ARG, "unknown dtype %d", (int)a.dtype);
+  if (a.batch < 0 || a.total_q < 0 || a.total_k < 0 || a.max_q < 0 || a.max_k < 0)
+    return fail(MXFA_ERR_INVALID_ARG, "negative size");
+  MXFA_TRY(check_heads(a.Hq, a.Hkv));
+  if (a.D != 64 && a.D != 128) return fail(MXFA_ERR_UNSUPPORTED, "head dim %d is not supported (64 or 128)", a.D);
+  if (std::isinf(a.scale)) return fail(MXFA_ERR_INVALID_ARG, "softmax_scale is infinite");
+  if (a.batch == 0 || a.total_q == 0) {
+    *noop = true;
+    return MXFA_OK;
+  }
+  if (!a.cu_q || !a.cu_k) return fail(MXFA_ERR_INVALID_ARG, "cu_seqlens_q / cu_seqlens_k is NULL");
+  if (a.max_q > a.total_q || a.max_k > a.total_k)
+    return fail(MXFA_ERR_INVALID_ARG, "max_seqlen exceeds the total token count");
+  MXFA_TRY(check_ptr(a.q, "q"));
+  MXFA_TRY(check_ptr(a.o, "o"));
+  MXFA_TRY(check_ptr(a.lse, "lse", true));
+  if (a.total_k > 0) {
+    MXFA_TRY(check_ptr(a.k, "k"));
+    MXFA_TRY(check_ptr(a.v, "v"));
+  }
+  return MXFA_OK;
+}
+
+// Strict mode: the cumulative lengths checked on the host (synchronises).
+mxfa_status_t varlen_strict(const VarlenArgs &a, cudaStream_t st) {
+  if (!strict_mode()) return MXFA_OK;
+  MXFA_TRY(strict_check_cu(a.cu_q, a.batch, a.total_q, a.max_q, "cu_seqlens_q", st));
+  return strict_check_cu(a.cu_k, a.batch, a.total_k, a.max_k, "cu_seqlens_k", st);
+}
+
+mxfa_status_t varlen_launch(const VarlenArgs &a, void *workspace, cudaStream_t st) {
+  AttnParams p{};
+  p.q = a.q; p.k = a.k; p.v = a.v; p.o = a.o; p.lse = a.lse;
+  p.cu_q = a.cu_q; p.cu_k = a.cu_k;
+  p.batch = a.batch; p.sq = 0; p.sk = 0; p.max_sq = a.max_q; p.max_sk = a.max_k;
+  p.hq = a.Hq; p.hkv = a.Hkv; p.dqk = a.D; p.dv = a.D;
+  p.q_rs = (int64_t)a.Hq * a.D; p.q_hs = a.D; p.k_rs = (int64_t)a.Hkv * a.D; p.k_hs = a.D;
+  p.v_rs = (int64_t)a.Hkv * a.D; p.v_hs = a.D; p.o_rs = (int64_t)a.Hq * a.D; p.o_hs = a.D;
+  p.scale_log2 = resolve_scale(a.scale, a.D) * kLog2e;
+  p.causal = a.causal ? 1 : 0;
+  p.hdr = static_cast<WsHeader *>(workspace);
+  p.pairs = nullptr;
+  p.wait_ns = g_wait_ns.load();
+  return prefill(p, a.dtype, a.D, true, a.total_q, a.total_k, workspace, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -524,6 +599,11 @@ extern "C" {
 const char *mxfa_last_error(void) { return g_err.c_str(); }
 
 uint32_t mxfa_version(void) { return (0u << 16) | (1u << 8) | 0u; }
+
+void mxfa_test_hooks(uint64_t wait_budget_ns, int keep_merge_counters) {
+  g_wait_ns.store(wait_budget_ns ? wait_budget_ns : kWaitBudgetNs);
+  g_keep_merge_counters.store(keep_merge_counters ? 1 : 0);
+}
 
 uint32_t mxfa_device_status_detail(void) { return g_detail; }
 
@@ -592,6 +672,7 @@ mxfa_status_t mxfa_attn_fwd(const void *q, const void *k, const void *v, void *o
   p.causal = causal ? 1 : 0;
   p.hdr = static_cast<WsHeader *>(workspace);
   p.pairs = nullptr;
+  p.wait_ns = g_wait_ns.load();
   return prefill(p, dtype, D, false, rows_q, rows_k, workspace, static_cast<cudaStream_t>(stream));
 }
 
@@ -600,42 +681,16 @@ mxfa_status_t mxfa_attn_varlen_fwd(const void *q, const void *k, const void *v, 
                                    int total_k, int max_seqlen_q, int max_seqlen_k, int Hq, int Hkv, int D,
                                    mxfa_dtype_t dtype, float softmax_scale, int causal, void *workspace,
                                    size_t workspace_bytes, void *stream) {
-  if (!dtype_ok(dtype)) return fail(MXFA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
-  if (batch < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
-    return fail(MXFA_ERR_INVALID_ARG, "negative size");
-  MXFA_TRY(check_heads(Hq, Hkv));
-  if (D != 64 && D != 128) return fail(MXFA_ERR_UNSUPPORTED, "head dim %d is not supported (64 or 128)", D);
-  if (std::isinf(softmax_scale)) return fail(MXFA_ERR_INVALID_ARG, "softmax_scale is infinite");
-  if (batch == 0 || total_q == 0) return MXFA_OK;
-  if (!cu_seqlens_q || !cu_seqlens_k) return fail(MXFA_ERR_INVALID_ARG, "cu_seqlens_q / cu_seqlens_k is NULL");
-  if (max_seqlen_q > total_q || max_seqlen_k > total_k)
-    return fail(MXFA_ERR_INVALID_ARG, "max_seqlen exceeds the total token count");
-  MXFA_TRY(check_ptr(q, "q"));
-  MXFA_TRY(check_ptr(o, "o"));
-  MXFA_TRY(check_ptr(lse, "lse", true));
-  if (total_k > 0) {
-    MXFA_TRY(check_ptr(k, "k"));
-    MXFA_TRY(check_ptr(v, "v"));
-  }
+  const VarlenArgs a{q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                     max_seqlen_k, Hq, Hkv, D, dtype, softmax_scale, causal};
+  bool noop = false;
+  MXFA_TRY(varlen_check(a, &noop));
+  if (noop) return MXFA_OK;
   MXFA_TRY(check_workspace(workspace, workspace_bytes,
                            mxfa_attn_varlen_fwd_workspace_size(batch, max_seqlen_q, max_seqlen_k, Hq, D, dtype)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (strict_mode()) {
-    MXFA_TRY(strict_check_cu(cu_seqlens_q, batch, total_q, max_seqlen_q, "cu_seqlens_q", st));
-    MXFA_TRY(strict_check_cu(cu_seqlens_k, batch, total_k, max_seqlen_k, "cu_seqlens_k", st));
-  }
-  AttnParams p{};
-  p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
-  p.cu_q = cu_seqlens_q; p.cu_k = cu_seqlens_k;
-  p.batch = batch; p.sq = 0; p.sk = 0; p.max_sq = max_seqlen_q; p.max_sk = max_seqlen_k;
-  p.hq = Hq; p.hkv = Hkv; p.dqk = D; p.dv = D;
-  p.q_rs = (int64_t)Hq * D; p.q_hs = D; p.k_rs = (int64_t)Hkv * D; p.k_hs = D;
-  p.v_rs = (int64_t)Hkv * D; p.v_hs = D; p.o_rs = (int64_t)Hq * D; p.o_hs = D;
-  p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
-  p.causal = causal ? 1 : 0;
-  p.hdr = static_cast<WsHeader *>(workspace);
-  p.pairs = nullptr;
-  return prefill(p, dtype, D, true, total_q, total_k, workspace, st);
+  MXFA_TRY(varlen_strict(a, st));
+  return varlen_launch(a, workspace, st);
 }
 
 size_t mxfa_attn_decode_splitkv_workspace_size(int batch, int max_q_len, int Hq, int Hkv, int Dv, int max_kv_len,
@@ -696,6 +751,7 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
   p.causal = causal ? 1 : 0;
   p.hdr = static_cast<WsHeader *>(workspace);
   p.pairs = nullptr;
+  p.wait_ns = g_wait_ns.load();
   if (decode_tc_eligible(dtype, Hq, Hkv, Dqk, Dv, max_q_len, k, v, k_row_stride, v_row_stride) && total_kv > 0)
     return launch_decode_tc(p, dtype, total_q, total_kv, num_splits, workspace, st);
   if (decode_gqa_eligible(dtype, Hq, Hkv, Dqk, Dv, max_q_len, k_row_stride, v_row_stride) && total_kv > 0) {
@@ -754,6 +810,7 @@ mxfa_status_t mxfa_attn_decode_mla_fp8kv(const void *q, const void *kv, float kv
   p.causal = causal ? 1 : 0;
   p.hdr = static_cast<WsHeader *>(workspace);
   p.pairs = nullptr;
+  p.wait_ns = g_wait_ns.load();
   return launch_decode_tc(p, MXFA_BF16, total_q, total_kv, num_splits, workspace, st, true, kv_scale);
 }
 
@@ -821,6 +878,7 @@ mxfa_status_t mxfa_attn_decode_kvcache(const void *q, void *k_cache, void *v_cac
   p.causal = causal ? 1 : 0;
   p.hdr = static_cast<WsHeader *>(workspace);
   p.pairs = nullptr;
+  p.wait_ns = g_wait_ns.load();
   int sms = 0;
   MXFA_TRY(sm_count(&sms));
   DecodeSched s = decode_sched(p, Hkv, num_splits, D, kGqKeys, workspace, sms);
@@ -886,8 +944,13 @@ extern "C" mxfa_status_t mxfa_attn_varlen_fwd_noalloc(const void *q, const void 
                                                       int total_k, int max_seqlen_q, int max_seqlen_k, int Hq,
                                                       int Hkv, int D, mxfa_dtype_t dtype, float softmax_scale,
                                                       int causal, void *stream) {
-  if (!dtype_ok(dtype)) return fail(MXFA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
-  if (batch < 0 || max_seqlen_q < 0 || max_seqlen_k < 0) return fail(MXFA_ERR_INVALID_ARG, "negative size");
+  const VarlenArgs a{q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                     max_seqlen_k, Hq, Hkv, D, dtype, softmax_scale, causal};
+  // Every argument check of mxfa_attn_varlen_fwd runs before the scratch
+  // array is touched, so a rejected call writes nothing.
+  bool noop = false;
+  MXFA_TRY(varlen_check(a, &noop));
+  if (noop) return MXFA_OK;
   const size_t need = mxfa_attn_varlen_fwd_workspace_size(batch, max_seqlen_q, max_seqlen_k, Hq, D, dtype);
   if (need > kNoAllocScratchBytes)
     return fail(MXFA_ERR_WORKSPACE,
@@ -896,10 +959,18 @@ extern "C" mxfa_status_t mxfa_attn_varlen_fwd_noalloc(const void *q, const void 
                 need, kNoAllocScratchBytes);
   void *scratch = nullptr;
   MXFA_TRY(noalloc_scratch(&scratch));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MXFA_TRY(varlen_strict(a, st));
   // The header (status word, unit count) must start at zero; the schedule
   // tables after it are fully rewritten by every call.
-  MXFA_CUDA(cudaMemsetAsync(scratch, 0, sizeof(WsHeader), static_cast<cudaStream_t>(stream)));
-  return mxfa_attn_varlen_fwd(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
-                              max_seqlen_k, Hq, Hkv, D, dtype, softmax_scale, causal, scratch, kNoAllocScratchBytes,
-                              stream);
+  MXFA_CUDA(cudaMemsetAsync(scratch, 0, sizeof(WsHeader), st));
+  return varlen_launch(a, scratch, st);
+}
+
+// The status word of the scratch array: what mxfa_read_device_status reads
+// from a caller's workspace, read here from the array of the current device.
+extern "C" mxfa_status_t mxfa_read_noalloc_status(void *stream) {
+  void *scratch = nullptr;
+  MXFA_TRY(noalloc_scratch(&scratch));
+  return mxfa_read_device_status(scratch, stream);
 }

@@ -20,19 +20,24 @@
 // more than 2^8.  Until then O and l keep the stale maximum as their common
 // base, which leaves O = acc / l and LSE = base + log2(l) exact.
 //
-// Roles (640 threads, five warpgroups):
+// Roles (768 threads, six warpgroups; launched at 80 registers per thread,
+// then setmaxnreg gives warpgroups 0 and 5 48 and warpgroups 1-4 96):
 //   warp 0      TMA producer: Q tiles once per unit, then K_j, V_j into a
 //               ring of shared-memory slots (128B-swizzled boxes of 64 cols)
 //   warp 1      TMEM allocator and MMA issuer: the whole warp runs the
 //               schedule and one elected lane issues; it alternates the two
 //               query tiles (PV_0(j), S_0(j+1), PV_1(j), S_1(j+1)) so one
 //               tile's softmax overlaps the other tile's MMAs
-//   warps 4-19  softmax + epilogue.  A query row has four threads, one per
-//               32-key group g = (warp-4)/4, in the four warps of its TMEM
+//   warps 2-3   idle (they complete warpgroup 0 for setmaxnreg)
+//   warps 4-19  softmax.  A query row has four threads, one per 32-key
+//               group g = (warp-4)/4, in the four warps of its TMEM
 //               sub-partition (warp w reads lanes 32*(w%4)..+31); these four
 //               warps take query tile 0 and query tile 1 in turn, and vote
 //               (bar.red.and) on whether the stale base still bounds every
 //               row before exchanging partial maxima through shared memory.
+//               At the end of a unit they hand the row sums and write LSE.
+//   warps 20-23 output epilogue: O_t / l in the output dtype, one thread per
+//               row, then O_t's TMEM columns go back to the MMA issuer.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
 //
 // Every wait is bounded (see wait_bar); a wait that runs out records
@@ -326,7 +331,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       for (int it = 0, u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
         const UnitInfo ui = unit_info(p, u);
         const int nmax = max(ui.n[0], ui.n[1]);
-        if (it > 0 && !wait_bar(b_qe, (it - 1) & 1, abort_flag, hdr, kSiteQEmpty)) break;
+        if (it > 0 && !wait_bar(b_qe, (it - 1) & 1, abort_flag, hdr, kSiteQEmpty, p.wait_ns)) break;
         mbar_arrive_expect_tx(b_qf, 2 * Cfg::kTileBytes);
         const int qrow = ui.sr.q0 + ui.m * kTcUnitRows;
 #pragma unroll
@@ -339,7 +344,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         for (int j = 0; j < nmax && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv, ++ring) {
             const int s = ring % Cfg::kSlots;
-            if (!wait_bar(b_se(s), ((ring / Cfg::kSlots) & 1) ^ 1, abort_flag, hdr, kSiteSlotEmpty)) {
+            if (!wait_bar(b_se(s), ((ring / Cfg::kSlots) & 1) ^ 1, abort_flag, hdr, kSiteSlotEmpty, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -356,12 +361,12 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       // CTA exits (on the normal path they were all consumed already).
       const uint64_t t0 = global_ns();
       if (q_issued > 0)
-        while (!mbar_test(b_qf, (q_issued - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        while (!mbar_test(b_qf, (q_issued - 1) & 1) && global_ns() - t0 < p.wait_ns) {
         }
       for (int s = 0; s < Cfg::kSlots; ++s) {
         const uint32_t uses = ring / Cfg::kSlots + ((uint32_t)s < ring % Cfg::kSlots ? 1u : 0u);
         if (uses == 0) continue;
-        while (!mbar_test(b_sf(s), (uses - 1) & 1) && global_ns() - t0 < kWaitBudgetNs) {
+        while (!mbar_test(b_sf(s), (uses - 1) & 1) && global_ns() - t0 < p.wait_ns) {
         }
       }
     }
@@ -372,7 +377,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     const bool leader = elect_one();
     // every lane waits; the warp gives up together if any lane gave up
     auto wait_warp = [&](uint32_t bar, uint32_t parity, volatile int *ab, WsHeader *h, uint32_t site) {
-      return __all_sync(0xffffffffu, wait_bar(bar, parity, ab, h, site));
+      return __all_sync(0xffffffffu, wait_bar(bar, parity, ab, h, site, p.wait_ns));
     };
     {
       constexpr uint32_t idesc_s = make_idesc_f16(BF16, kTcBlockM, kTcBlockN, false, false);
@@ -481,7 +486,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       // Teardown: all MMAs issued by the elected lane complete before TMEM is freed.
       if (leader) mma_commit(smem_u32(&ctrl->drain));
       const uint64_t t0 = global_ns();
-      while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < kWaitBudgetNs) {
+      while (!mbar_test(smem_u32(&ctrl->drain), 0) && global_ns() - t0 < p.wait_ns) {
       }
     }
   }
@@ -512,7 +517,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         // the exchange area holds the previous unit's row sums until the
         // epilogue warpgroup has taken them
         bool lf = true;
-        if (it > 0) lf = wait_bar(smem_u32(&ctrl->l_free), (it - 1) & 1, abort_flag, hdr, kSiteLFree);
+        if (it > 0) lf = wait_bar(smem_u32(&ctrl->l_free), (it - 1) & 1, abort_flag, hdr, kSiteLFree, p.wait_ns);
         __syncwarp();
         if (bar_or(bar_id, 128, !__all_sync(0xffffffffu, lf))) break;
       }
@@ -528,7 +533,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
           // A failed wait does not leave the loop here: the four warps of the
           // sub-partition first agree on it at the next named barrier, so
           // none is left waiting there for a warp that has gone.
-          const bool got_s = wait_bar(smem_u32(&ctrl->s_full[t]), s_cnt[t] & 1, abort_flag, hdr, kSiteSFull);
+          const bool got_s = wait_bar(smem_u32(&ctrl->s_full[t]), s_cnt[t] & 1, abort_flag, hdr, kSiteSFull, p.wait_ns);
           __syncwarp();
           const bool wok = __all_sync(0xffffffffu, got_s);
           ++s_cnt[t];
@@ -632,7 +637,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     bool ok = true;
     for (int it = 0, u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
       const UnitInfo ui = unit_info(p, u);
-      const bool got_l = wait_bar(smem_u32(&ctrl->l_ready), it & 1, abort_flag, hdr, kSiteLReady);
+      const bool got_l = wait_bar(smem_u32(&ctrl->l_ready), it & 1, abort_flag, hdr, kSiteLReady, p.wait_ns);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got_l)) break;
       const float lt0 = ctrl->xchg[0][r], lt1 = ctrl->xchg[1][r];
@@ -645,7 +650,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         const bool valid = i < ui.sr.sq;
         T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(ui.sr.q0 + i) * p.o_rs + (int64_t)ui.h * p.o_hs;
         if (ui.n[t] > 0) {
-          const bool got_o = wait_bar(smem_u32(&ctrl->o_done[t]), o_cnt[t] & 1, abort_flag, hdr, kSiteODone);
+          const bool got_o = wait_bar(smem_u32(&ctrl->o_done[t]), o_cnt[t] & 1, abort_flag, hdr, kSiteODone, p.wait_ns);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got_o)) {
             ok = false;

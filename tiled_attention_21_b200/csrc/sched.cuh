@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(kPrepThreads)
 prefill_prep_kernel(const AttnParams p, int *prefix, int *bucket, int n_buckets, int2 *pairs, int max_pairs) {
   using Scan = cub::BlockScan<int, kPrepThreads>;
   __shared__ typename Scan::TempStorage tmp;
-  __shared__ int carry;
+  __shared__ int carry, n_blocks;
   const int tid = threadIdx.x;
   if (tid == 0) carry = 0;
   for (int i = tid; i < n_buckets; i += kPrepThreads) bucket[i] = 0;
@@ -62,9 +62,12 @@ prefill_prep_kernel(const AttnParams p, int *prefix, int *bucket, int n_buckets,
     if (tid == 0) carry += total;
     __syncthreads();
   }
-  if (tid == 0) prefix[0] = 0;
-  const int n_pairs = min(carry, max_pairs);
+  if (tid == 0) {
+    prefix[0] = 0;
+    n_blocks = carry;  // every (sequence, 256-row block) pair, before the clamp to the schedule's room
+  }
   __syncthreads();
+  const int n_pairs = min(n_blocks, max_pairs);
 
   // histogram over key = (n_buckets - 1 - cost): descending cost
   for (int idx = tid; idx < n_pairs; idx += kPrepThreads) {
@@ -95,7 +98,9 @@ prefill_prep_kernel(const AttnParams p, int *prefix, int *bucket, int n_buckets,
   }
   if (tid == 0) {
     p.hdr->n_units = (uint32_t)n_pairs;
-    if (carry > max_pairs) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x201);
+    // A sequence longer than the max_seqlen_q the schedule was sized for
+    // leaves blocks unscheduled: their rows of O would never be written.
+    if (n_blocks > max_pairs) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x201);
   }
 }
 

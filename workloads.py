@@ -289,6 +289,19 @@ def cfg_long_causal(S: int = 32768, H: int = 32, rows_per_head: int = 256) -> Pr
                    meta={"B": 1, "Sq": S, "Sk": S})
 
 
+def to_device(p: Problem, device="cuda") -> dict:
+    """The problem's tensors copied to `device` (a plain copy, no arithmetic):
+    q, k, v, cu_q, cu_k, and for MLA decode the one kv cache with k and v as
+    its [total, 1, 576] and [total, 1, 512] views."""
+    d = {"q": p.q.to(device), "k": p.k.to(device), "v": p.v.to(device),
+         "cu_q": p.cu_q.to(device), "cu_k": p.cu_k.to(device)}
+    if p.mla:
+        d["kv"] = p.kv.to(device)
+        d["k"] = d["kv"].view(-1, 1, p.dqk)
+        d["v"] = d["kv"][:, :p.dv].view(-1, 1, p.dv)
+    return d
+
+
 def sample_rows(p: Problem, n_per_head: int, seed: int) -> torch.Tensor:
     """(token, head) pairs for a sampled oracle check: n random tokens per head,
     plus the first and last token of every sequence."""
