@@ -168,14 +168,20 @@ mxfa_status_t mxfa_read_noalloc_status(void *stream);
  * Dqk = 576, Dv = 512, k_row_stride = v_row_stride = 576: value = first 512
  * columns of each cached row; the tensor-core kernel reads each KV tile once
  * and uses it as both operands.  That path needs bf16/f16 and
- * max_q_len * Hq <= 64.
+ * max_q_len <= 64.
  * Grouped-query decode (mxflashattn flash_attn_with_kvcache shape): Dqk = Dv
- * = 64 or 128, bf16/f16, max_q_len * (Hq / Hkv) <= 64 and row strides that
- * are multiples of 8 elements run on the tensor-core kernel, which streams
- * each KV head once for the Hq / Hkv query heads that share it.  Other shapes
- * (or f32) run on the exact CUDA-core kernel.
+ * = 64 or 128, bf16/f16, max_q_len <= 64 and row strides that are multiples
+ * of 8 elements run on the tensor-core kernel, which streams each KV head
+ * once for the Hq / Hkv query heads that share it.  Other shapes (or f32)
+ * run on the exact CUDA-core kernel.
+ * Both tensor-core kernels compute 64 query rows (token, head) per pass over
+ * a KV head: when max_q_len * Hq / Hkv exceeds 64, the query heads of each KV
+ * head are split into the fewest equal groups of at most 64 rows (e.g. MLA
+ * q_len 8 x 16 heads: two groups of 8 heads), and each group streams the KV
+ * head again (the groups of one sequence run at about the same time, so the
+ * repeated reads mostly come from L2).
  * The workspace size takes Hkv because the grouped-query kernel schedules
- * batch * Hkv decode sequences.
+ * batch * Hkv * groups decode sequences.
  * num_splits: 0 = automatic: one run of KV tiles per SM, either whole
  *   sequences dealt out in order or the KV of all sequences cut into
  *   near-equal pieces, whichever balances better once the cost of merging a
@@ -217,8 +223,10 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
  *   q: [total_q, Hq, 576] bf16 contiguous; o: [total_q, Hq, 512] bf16;
  *   lse: [total_q, Hq] fp32 (or NULL); qo_indptr / kv_indptr, max lengths,
  *   causal, num_splits and the workspace as for mxfa_attn_decode_splitkv.
- *   Requires max_q_len * Hq <= 64 (else MXFA_ERR_UNSUPPORTED).  kv must be
- *   a valid 16-byte aligned pointer even when total_kv = 0.
+ *   Requires max_q_len <= 64 (else MXFA_ERR_UNSUPPORTED); more than 64
+ *   query rows per sequence are split into head groups as for
+ *   mxfa_attn_decode_splitkv.  kv must be a valid 16-byte aligned pointer
+ *   even when total_kv = 0.
  * The kernel widens each staged tile of codes to bf16 exactly in shared
  * memory and applies kv_scale to the scores and to the outputs, so the
  * result equals attention over the dequantised cache up to the bf16 path's
@@ -236,7 +244,8 @@ mxfa_status_t mxfa_attn_decode_mla_fp8kv(const void *q, const void *kv, float kv
  * flash_attn_with_kvcache: q, k_cache, v_cache, k, v, cache_seqlens,
  * block_table, causal).
  *   q: [batch, Sq, Hq, D] contiguous, bf16 or f16, D = 64 or 128,
- *      Sq * (Hq / Hkv) <= 64 (otherwise MXFA_ERR_UNSUPPORTED).
+ *      Sq <= 64 (otherwise MXFA_ERR_UNSUPPORTED; Sq * Hq / Hkv above 64 is
+ *      split into head groups as for mxfa_attn_decode_splitkv).
  *   k_cache, v_cache: [num_pages, page_size, Hkv, D] contiguous.  Dense cache
  *      (block_table == NULL): num_pages = batch, page_size = the cache length,
  *      key position pos of batch entry b is row b*page_size + pos.  Paged

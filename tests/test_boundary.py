@@ -107,7 +107,7 @@ def test_fp8_decode_validation(lib):
                                               a["tq"], a["tkv"], a["mq"], a["mkv"], a["Hq"], a["rs"], a["scale"],
                                               a["causal"], a["splits"], a["ws"], a["wn"], None)
 
-    assert c(Hq=32) == m.MXFA_ERR_UNSUPPORTED               # 4 x 32 query rows per sequence > 64
+    assert c(mq=65, tq=130) == m.MXFA_ERR_UNSUPPORTED      # more than 64 queries per sequence
     assert c(ks=float("inf")) == m.MXFA_ERR_INVALID_ARG     # scale not finite
     assert c(ks=float("nan")) == m.MXFA_ERR_INVALID_ARG
     assert c(rs=560) == m.MXFA_ERR_INVALID_ARG              # row shorter than 576 codes
@@ -119,6 +119,10 @@ def test_fp8_decode_validation(lib):
     assert c(B=0) == m.MXFA_OK                              # nothing to do
     need = lib.mxfa_attn_decode_mla_fp8kv_workspace_size(128, 4, 16, 8192, 0)
     assert need > 256 and need == lib.mxfa_attn_decode_splitkv_workspace_size(128, 4, 16, 1, 512, 8192, 0, 2)
+    # 8 x 16 query rows: two head groups, each a decode sequence of its own
+    need8 = lib.mxfa_attn_decode_mla_fp8kv_workspace_size(128, 8, 16, 8192, 0)
+    assert need8 > need and need8 == lib.mxfa_attn_decode_splitkv_workspace_size(128, 8, 16, 1, 512, 8192, 0, 2)
+    assert lib.mxfa_attn_decode_mla_fp8kv_workspace_size(128, 65, 16, 8192, 0) == 256
 
 
 def test_workspace_sizes(lib):
@@ -160,7 +164,7 @@ def test_kvcache_validation(lib):
 
     assert c(D=96) == m.MXFA_ERR_UNSUPPORTED                 # head dim
     assert c(dt=0) == m.MXFA_ERR_UNSUPPORTED                 # fp32
-    assert c(Sq=16) == m.MXFA_ERR_UNSUPPORTED                # 16 * 8 query rows per KV head > 64
+    assert c(Sq=65) == m.MXFA_ERR_UNSUPPORTED                # more than 64 queries per sequence
     assert c(page=48) == m.MXFA_ERR_UNSUPPORTED              # page size
     assert c(Hq=30) == m.MXFA_ERR_INVALID_ARG                # Hq not a multiple of Hkv
     assert c(Snew=2) == m.MXFA_ERR_INVALID_ARG               # appended rows without k_new / v_new

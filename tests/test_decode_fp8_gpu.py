@@ -107,11 +107,18 @@ def test_fp8_full_size_sampled_rows():
 
 def test_fp8_rejects_unsupported_shapes():
     import tiled_attention_21_b200 as mx
-    p = workloads.mla_decode_fp8(48, batch=2, q_len=8, kv_len=64, heads=16)  # 128 query rows
+    p = workloads.mla_decode_fp8(48, batch=2, q_len=65, kv_len=64, heads=2)  # more than 64 queries
     d = to_dev(p)
     with pytest.raises(mx.MxfaError) as e:
         run(p, d, "decode")
     assert e.value.status == mx.MXFA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kv_len,splits", [(300, 0), (300, 3), (8192, 0)])
+def test_fp8_q8_head_groups(kv_len, splits):
+    # 8 queries x 16 heads = 128 query rows: two groups of 8 heads on the tensor cores
+    p = workloads.mla_decode_fp8(49, batch=3, q_len=8, kv_len=kv_len, causal=True)
+    check(p, splits)
 
 
 def test_fp8_padded_cache_rows():

@@ -141,8 +141,31 @@ def test_gqa_tc_group_sizes():
 
 
 def test_gqa_rows_beyond_tensor_core_limit():
-    # q_len * G = 128 > 64 rows: the exact CUDA-core kernel takes it
-    check(workloads.gqa_decode(37, batch=2, q_len=16, kv_len=200, causal=True))
+    # more than 64 queries per sequence: the exact CUDA-core kernel takes it
+    check(workloads.gqa_decode(37, batch=2, q_len=70, kv_len=200, hq=4, hkv=4, causal=True))
+
+
+@pytest.mark.parametrize("q_len,hq,hkv,causal", [(16, 32, 4, True), (4, 32, 1, False), (3, 48, 2, True),
+                                                 (64, 8, 4, True)])
+def test_gqa_tc_head_groups(q_len, hq, hkv, causal):
+    # q_len * Hq/Hkv = 128, 128, 72 and 128 rows per KV head: the query heads
+    # of each KV head split into two groups (of 4, 16, 12 and 1 heads) on the
+    # tensor cores
+    p = workloads.gqa_decode(39, batch=3, q_len=q_len, kv_len=700, hq=hq, hkv=hkv, causal=causal)
+    check(p)
+    check(p, 3)
+
+
+@pytest.mark.parametrize("batch,kv_len,splits", [(3, 700, 0), (3, 700, 2), (2, 40000, 0), (200, 300, 0)])
+def test_mla_q8_head_groups(batch, kv_len, splits):
+    # 8 queries x 16 heads = 128 query rows: two groups of 8 heads, each
+    # streaming the latent cache; one launch (small), three kernels (a long
+    # sequence, or more sequences than SMs)
+    p = workloads.mla_decode(29, batch=batch, q_len=8, kv_len=kv_len)
+    if batch * 8 * 16 * kv_len > 50_000_000:
+        check(p, splits, workloads.sample_rows(p, 8, 7))
+    else:
+        check(p, splits)
 
 
 def test_gqa_tc_split_invariance():

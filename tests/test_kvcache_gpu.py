@@ -72,6 +72,12 @@ def test_append_single_token_gqa16_d64():
     run_case(w)
 
 
+def test_head_groups_sq16():
+    # 16 queries x 8 heads per KV head = 128 rows: two head groups per KV head
+    w = workloads.kvcache(48, batch=2, Sq=16, Snew=16, seqlens=[100, 300], page_size=64, causal=True)
+    run_case(w, causal=True)
+
+
 def test_split_invariance():
     w = workloads.kvcache(45, batch=2, Sq=1, Snew=0, seqlens=[3000, 4096], page_size=128)
     o1, l1 = run_case(w, num_splits=1)

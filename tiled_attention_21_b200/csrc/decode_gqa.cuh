@@ -3,12 +3,14 @@
 //
 // Shape (the flash_attn_with_kvcache decode of mxflashattn 1.4.0 api.py and
 // the q_len = 1 decode bench of AstrAI attn_decode_split_kv_mma.cuh): Hq
-// query heads in Hkv groups of G = Hq/Hkv, one K and one V head per group,
-// head dim D in {64, 128}, q_len*G <= 64.  The decode "sequence" v of the
-// split schedule (decode_prep_kernel) is (batch entry b, KV head g); its
-// q_len*G query rows, flattened r = q*G + j for token q and head g*G + j,
-// form the M = 64 side of every MMA (rows past q_len*G are zero and never
-// stored).
+// query heads in Hkv groups of Hq/Hkv, one K and one V head per group, head
+// dim D in {64, 128}, q_len <= 64.  The decode "sequence" v of the split
+// schedule (decode_prep_kernel) is (batch entry b, head group gh): G = Hq /
+// heads query heads gh*G .. gh*G+G-1 that read KV head gh / subs, with
+// q_len*G <= 64 (subs = 1, one group per KV head, whenever q_len*Hq/Hkv <=
+// 64).  Its q_len*G query rows, flattened r = q*G + j for token q and head
+// gh*G + j, form the M = 64 side of every MMA (rows past q_len*G are zero and
+// never stored).
 //
 // The K and V heads of each sequence are streamed exactly once: 128-key
 // tiles arrive by TMA as D/64 column chunks of K followed by D/64 chunks of
@@ -124,7 +126,8 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
       bool ok = true;
       for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
         const int4 sd = dc_seg(p, s, sg);
-        const int b = sd.x / s.heads, g = sd.x % s.heads;
+        const DcSeq sq = dc_seq(p, s, sd.x);
+        const int b = sq.b, g = sq.kvh;
         const int len = dc_klen(p, s, b);
         for (int j = sd.y; ok && j < sd.z; ++j, ++tc) {
           const int x = tc % Cfg::kRingTiles;
@@ -248,7 +251,8 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     // Q rows of piece sg into TMEM (lanes 16-31, columns kGqQCol..): this
     // thread writes half `half` of row r.
     auto load_q = [&](int sg) {
-      const int v = dc_seg(p, s, sg).x, b = v / s.heads, gh = v % s.heads;
+      const DcSeq ds = dc_seq(p, s, dc_seg(p, s, sg).x);
+      const int b = ds.b, gh = ds.gh;
       const int q0 = dc_q(p, b).x, rows = dc_q(p, b).y * G;
       const bool vq = r < rows;
       const uint4 *src = reinterpret_cast<const uint4 *>(
@@ -271,7 +275,9 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     if (seg_lo < seg_hi) load_q(seg_lo);
     for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
       const int4 sd = dc_seg(p, s, sg);
-      const int v = sd.x, b = v / s.heads, gh = v % s.heads;
+      const int v = sd.x;
+      const DcSeq ds = dc_seq(p, s, v);
+      const int b = ds.b, gh = ds.gh;
       const int q0 = dc_q(p, b).x, sq = dc_q(p, b).y, sk = dc_klen(p, s, b);
       const int rows = sq * G;
       const bool valid = r < rows;

@@ -3,8 +3,10 @@
 // Shape (kernelbot-amd-mixed-mla submission 588924, _flash_fused /
 // _flash_splitk / _reduce_splitk): every sequence b has q_len queries of Hq
 // heads that all read one shared latent KV row of 576 columns; the value is
-// the first 512 columns of that same row.  The q_len*Hq <= 64 query rows of a
-// sequence are flattened r = q*Hq + h and form the M = 64 side of every MMA.
+// the first 512 columns of that same row.  The query heads are taken in head
+// groups of G heads with q_len*G <= 64 (one group, G = Hq, when q_len*Hq <=
+// 64); the q_len*G query rows of a group are flattened r = q*G + j (token q,
+// head gh*G + j) and form the M = 64 side of every MMA.
 //
 // The KV cache is streamed exactly once: 64-key tiles arrive by TMA as nine
 // 8 KB column chunks (64 keys x 64 columns, 128B swizzle) into a 27-slot
@@ -56,11 +58,19 @@ constexpr int kDcSmemBytes = kDcCtrlBytes + kDcSlots * kDcChunkBytes + kDcRows *
 static_assert(kDcSmemBytes <= 232448, "shared memory budget");
 constexpr int kDcMaxGrid = 256;
 
-// A decode "sequence" v is (batch entry b, KV head g) = (v / heads, v % heads):
-// heads = 1 for MLA (all query heads share the one latent KV head), Hkv for
-// grouped-query decode (the G = Hq/Hkv query heads of KV head g).
+// A decode "sequence" v is (batch entry b, head group gh) (dc_seq): the
+// G = Hq/heads query heads gh*G .. gh*G+G-1 of b, which read KV head
+// gh / subs.  heads = Hkv * subs: 1 for MLA (all query heads share the one
+// latent KV head), Hkv for grouped-query decode (the query heads of KV head
+// g); subs > 1 splits each KV head's query heads into subs groups when
+// q_len * Hq/Hkv exceeds the 64 query rows of the MMAs.  Each group streams
+// the KV head again; the sequences are numbered group-major (all batch
+// entries of group 0, then of group 1, ...), so the groups of one batch
+// entry land on CTAs far apart in the tile order and read the same tiles at
+// about the same time, the later reads from L2.
 struct DecodeSched {
-  int heads;       // KV heads per batch entry that form separate sequences
+  int heads;       // head groups per batch entry that form separate sequences
+  int subs;        // head groups per KV head
   int keys;        // keys per KV tile
   int *n_tiles;    // [batch*heads] KV tiles per sequence
   int *tile_pre;   // [batch*heads + 1] prefix of n_tiles
@@ -102,6 +112,21 @@ struct DecodeSched {
   // scale is folded into AttnParams::scale_log2 by the host).
   float o_scale;
 };
+
+struct DcSeq {
+  int b, gh, kvh;  // batch entry, head group, KV head
+};
+// v = (sub * batch + b) * Hkv + kvh with gh = kvh * subs + sub.
+__device__ __forceinline__ DcSeq dc_seq(const AttnParams &p, const DecodeSched &s, int v) {
+  const int hkv = s.heads / s.subs;
+  const int n_bh = p.batch * hkv;
+  const int sub = v / n_bh, w = v - sub * n_bh;
+  DcSeq r;
+  r.b = w / hkv;
+  r.kvh = w - r.b * hkv;
+  r.gh = r.kvh * s.subs + sub;
+  return r;
+}
 
 // Queries of batch entry b: (first row, count); packed (cu_q) or uniform.
 __device__ __forceinline__ int2 dc_q(const AttnParams &p, int b) {
@@ -176,7 +201,7 @@ __device__ __forceinline__ float4 *dc_pacc(const DecodeSched &s, int sg, int r, 
 
 // KV tiles of decode sequence v (0 when its batch entry has no query).
 __device__ __forceinline__ int dc_seq_tiles(const AttnParams &p, const DecodeSched &s, int v) {
-  const int b = v / s.heads;
+  const int b = dc_seq(p, s, v).b;
   if (dc_q(p, b).y <= 0) return 0;
   return (dc_klen(p, s, b) + s.keys - 1) / s.keys;
 }
@@ -231,7 +256,8 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     const int b = base + tid;
     int n = 0;
     if (b < B) {
-      const int e = b / s.heads;  // batch entry of sequence b
+      const DcSeq sq_b = dc_seq(p, s, b);
+      const int e = sq_b.b;  // batch entry of sequence b
       int len = p.cu_k ? p.cu_k[e + 1] - p.cu_k[e] : s.cache_seqlens[e] + s.add;
       if (!p.cu_k) {
         // A cache entry holds at most page_size keys (dense) or max_blocks
@@ -239,10 +265,10 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
         // no page at all, so the length is cut there and the call reports it.
         const int64_t cap = s.block_table ? (int64_t)s.max_blocks * s.page_size : (int64_t)s.page_size;
         if (len > cap) {
-          if (b % s.heads == 0) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x402);
+          if (sq_b.gh == 0) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x402);
           len = (int)cap;
         }
-        if (b % s.heads == 0) s.kv_len[e] = len;
+        if (sq_b.gh == 0) s.kv_len[e] = len;
       }
       n = (len + s.keys - 1) / s.keys;
       if (dc_q(p, e).y <= 0) n = 0;  // no queries: nothing to compute
@@ -376,7 +402,8 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
 template <typename T, int DV, int NT>
 __device__ void dc_merge_pieces(const AttnParams &p, const DecodeSched &s, int v, int i, int k, float *scratch) {
   volatile int *flag = reinterpret_cast<volatile int *>(scratch);
-  const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
+  const DcSeq sq = dc_seq(p, s, v);
+  const int b = sq.b, gh = sq.gh, G = p.hq / s.heads;
   const int2 qr = dc_q(p, b);
   const int rows = qr.y * G;
   // scratch: flag, then per row M and L, then the weights w and sums l of
@@ -479,7 +506,8 @@ __device__ void dc_merge_pieces(const AttnParams &p, const DecodeSched &s, int v
 // gets O = 0 and LSE = -inf, written by its CTA 0.
 template <typename T, int DV, int NT>
 __device__ void dc_zero_rows(const AttnParams &p, const DecodeSched &s, int v) {
-  const int b = v / s.heads, gh = v % s.heads, G = p.hq / s.heads;
+  const DcSeq sq = dc_seq(p, s, v);
+  const int b = sq.b, gh = sq.gh, G = p.hq / s.heads;
   const int2 qr = dc_q(p, b);
   const int rows = qr.y * G;
   for (int it = threadIdx.x; it < rows * DV; it += NT) {
@@ -606,9 +634,9 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       bool ok = true;
       for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
         const int4 sd = dc_seg(p, s, sg);
-        const int k0 = p.cu_k[sd.x];
-        if (sg + 1 < seg_hi) {  // the next piece's query rows, into L2
-          const int bn = dc_seg(p, s, sg + 1).x;
+        const int k0 = p.cu_k[dc_seq(p, s, sd.x).b];
+        if (sg + 1 < seg_hi) {  // the next piece's query tokens (all heads), into L2
+          const int bn = dc_seq(p, s, dc_seg(p, s, sg + 1).x).b;
           const int64_t q0n = p.cu_q[bn], rn = (p.cu_q[bn + 1] - q0n) * p.hq;
           if (rn > 0)
             tma_prefetch_bytes(reinterpret_cast<const uint16_t *>(p.q) + q0n * p.hq * kDcDqk,
@@ -826,13 +854,15 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     const uint32_t s_row = tmem + ((uint32_t)(sub * 32 + 16) << 16);
     const float c = p.scale_log2;
     const bool neg = c < 0.f;
+    const int G = p.hq / s.heads;  // query heads per sequence: row r is token r / G, head gh*G + r % G
     // Q rows of piece sg into TMEM (lanes 16-31, columns kDcQCol..): this
     // thread writes half `half` of row r; all global loads are issued first.
     auto load_q = [&](int sg) {
-      const int bq = dc_seg(p, s, sg).x;
-      const int q0 = p.cu_q[bq], rows = (p.cu_q[bq + 1] - q0) * p.hq;
+      const DcSeq sq_q = dc_seq(p, s, dc_seg(p, s, sg).x);
+      const int bq = sq_q.b, ghq = sq_q.gh;
+      const int q0 = p.cu_q[bq], rows = (p.cu_q[bq + 1] - q0) * G;
       const uint4 *src = reinterpret_cast<const uint4 *>(
-          reinterpret_cast<const uint16_t *>(p.q) + ((int64_t)q0 * p.hq + r) * kDcDqk);
+          reinterpret_cast<const uint16_t *>(p.q) + ((int64_t)(q0 + r / G) * p.hq + ghq * G + r % G) * kDcDqk);
       const bool vq = r < rows;
 #pragma unroll
       for (int k2 = 0; k2 < 2; ++k2) {
@@ -867,11 +897,12 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     if (seg_lo < seg_hi) load_q(seg_lo);
     for (int sg = seg_lo; ok && sg < seg_hi; ++sg) {
       const int4 sd = dc_seg(p, s, sg);
-      const int b = sd.x;
+      const DcSeq sq_v = dc_seq(p, s, sd.x);
+      const int b = sq_v.b, gh = sq_v.gh;
       const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0, sk = p.cu_k[b + 1] - p.cu_k[b];
-      const int rows = sq * p.hq;
+      const int rows = sq * G;
       const bool valid = r < rows;
-      const int nv = valid ? visible_keys(r / p.hq, sq, sk, p.causal) : 0;
+      const int nv = valid ? visible_keys(r / G, sq, sk, p.causal) : 0;
       float m_used = -INFINITY, l = 0.f;
       for (int j = sd.y; j < sd.z; ++j, ++g) {
         const bool got = wait_bar(b_sf, g & 1, abort_flag, hdr, kDSiteSFull, p.wait_ns);
@@ -966,8 +997,8 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         if (!__all_sync(0xffffffffu, got_o)) break;
         tc_fence_after();
       }
-      const bool direct = dc_seg_cnt(p, s, b) == 1;
-      const int tok = q0 + (valid ? r / p.hq : 0), h = valid ? r % p.hq : 0;
+      const bool direct = dc_seg_cnt(p, s, sd.x) == 1;
+      const int tok = q0 + (valid ? r / G : 0), h = gh * G + (valid ? r % G : 0);
       using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
       const float inv = l > 0.f ? (FP8 ? s.o_scale : 1.f) / l : 0.f;
 #pragma unroll 1
@@ -1054,7 +1085,8 @@ __global__ void __launch_bounds__(kDcCombineThreads) decode_combine_kernel(const
     // not split: stored directly by the decode kernel (a sequence with no
     // piece, cnt = 0, is written here: O = 0, LSE = -inf)
     if (cnt == 1) continue;
-    const int b = v / s.heads, gh = v % s.heads;
+    const DcSeq sq = dc_seq(p, s, v);
+    const int b = sq.b, gh = sq.gh;
     const int2 qr = dc_q(p, b);
     if (r >= qr.y * G) continue;
     const int base = s.seg_base[v];

@@ -372,26 +372,40 @@ DecodeWs decode_ws(int batch, int max_kv_len, int num_splits, int dv, int keys) 
   return w;
 }
 
+// Head groups per KV head of the tensor-core decode kernels: the smallest
+// divisor d of the G query heads sharing a KV head with max_q_len * G / d
+// <= 64 query rows per decode sequence (the M side of their MMAs); 0 when
+// there is none (max_q_len > 64).
+int head_subgroups(int G, int max_q_len) {
+  if (max_q_len <= 0) return 1;
+  for (int d = 1; d <= G; ++d)
+    if (G % d == 0 && (int64_t)max_q_len * (G / d) <= kDcRows) return d;
+  return 0;
+}
+
 bool decode_tc_eligible(mxfa_dtype_t dt, int Hq, int Hkv, int Dqk, int Dv, int max_q_len, const void *k,
                         const void *v, int64_t k_rs, int64_t v_rs) {
   return dt != MXFA_F32 && Dqk == kDcDqk && Dv == kDcDv && Hkv == 1 && k == v && k_rs == v_rs &&
-         (int64_t)max_q_len * Hq <= kDcRows;
+         head_subgroups(Hq, max_q_len) > 0;
 }
 
 // The grouped-query tensor-core decode: K and V heads of dimension 64 or 128,
-// 16-bit, q_len x G <= 64 query rows per KV head, rows TMA-addressable.
+// 16-bit, at most 64 queries per sequence, rows TMA-addressable.
 bool decode_gqa_eligible(mxfa_dtype_t dt, int Hq, int Hkv, int Dqk, int Dv, int max_q_len, int64_t k_rs,
                          int64_t v_rs) {
-  return dt != MXFA_F32 && Dqk == Dv && (Dqk == 64 || Dqk == 128) && (int64_t)max_q_len * (Hq / Hkv) <= kDcRows &&
+  return dt != MXFA_F32 && Dqk == Dv && (Dqk == 64 || Dqk == 128) && head_subgroups(Hq / Hkv, max_q_len) > 0 &&
          (k_rs * 2) % 16 == 0 && (v_rs * 2) % 16 == 0;
 }
 
-// Split schedule in the workspace for `heads` decode sequences per batch entry.
-DecodeSched decode_sched(const AttnParams &p, int heads, int num_splits, int dv, int keys, void *ws, int sms) {
+// Split schedule in the workspace for `heads` = Hkv * subs decode sequences
+// (head groups) per batch entry.
+DecodeSched decode_sched(const AttnParams &p, int heads, int subs, int num_splits, int dv, int keys, void *ws,
+                         int sms) {
   const DecodeWs w = decode_ws(p.batch * heads, p.max_sk, num_splits, dv, keys);
   char *base = static_cast<char *>(ws);
   DecodeSched s;
   s.heads = heads;
+  s.subs = subs;
   s.keys = keys;
   s.n_tiles = reinterpret_cast<int *>(base + w.n_tiles);
   s.tile_pre = reinterpret_cast<int *>(base + w.tile_pre);
@@ -437,7 +451,7 @@ mxfa_status_t launch_decode_gqa_t(AttnParams &p, const DecodeSched &s, mxfa_dtyp
   MXFA_TRY(make_map(&mv, p.v, dt, D, p.hkv, kv_rows, p.v_rs, p.v_hs, box));
   auto k = attn_decode_gqa_kernel<D, BF16>;
   // Small problems on packed K/V run in one launch, as for the MLA kernel.
-  const int n_seq = p.batch * p.hkv, max_tiles = (p.max_sk + kGqKeys - 1) / kGqKeys;
+  const int n_seq = p.batch * s.heads, max_tiles = (p.max_sk + kGqKeys - 1) / kGqKeys;
   if (s.num_splits == 0 && p.cu_k && n_seq <= s.grid && (int64_t)n_seq * max_tiles <= 4 * (int64_t)s.grid) {
     DecodeSched sa = s;
     const int t_min = max_tiles > 16 ? 4 : 2;  // tiles per piece at least (merge cost vs chain length)
@@ -482,8 +496,10 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
                                cudaStream_t st, bool kv_fp8 = false, float o_scale = 1.f) {
   int sms = 0;
   MXFA_TRY(sm_count(&sms));
-  DecodeSched s = decode_sched(p, 1, num_splits, kDcDv, kDcKeys, ws, sms);
+  const int subs = head_subgroups(p.hq, p.max_sq);
+  DecodeSched s = decode_sched(p, subs, subs, num_splits, kDcDv, kDcKeys, ws, sms);
   s.o_scale = o_scale;
+  const int n_seq = p.batch * subs;  // decode sequences: (batch entry, head group)
   CUtensorMap mq, mkv;
   MXFA_TRY(make_map_2d(&mq, p.q, dt, kDcDqk, (int64_t)total_q * p.hq, kDcDqk));
   if (kv_fp8)
@@ -498,22 +514,22 @@ mxfa_status_t launch_decode_tc(AttnParams &p, mxfa_dtype_t dt, int total_q, int 
   // Small problems run in one launch: no prep kernel (the pieces follow from
   // kv_indptr) and no combine kernel (split sequences merge in the kernel).
   const int max_tiles = (p.max_sk + kDcKeys - 1) / kDcKeys;
-  if (num_splits == 0 && p.batch <= s.grid && (int64_t)p.batch * max_tiles <= 4 * (int64_t)s.grid) {
+  if (num_splits == 0 && n_seq <= s.grid && (int64_t)n_seq * max_tiles <= 4 * (int64_t)s.grid) {
     DecodeSched sa = s;
     const int t_min = max_tiles > 32 ? 4 : 2;  // tiles per piece at least (merge cost vs chain length)
-    sa.arith_k = std::max(1, std::min(s.grid / p.batch, (max_tiles + t_min - 1) / t_min));
+    sa.arith_k = std::max(1, std::min(s.grid / n_seq, (max_tiles + t_min - 1) / t_min));
     if (sa.arith_k > 1 && !g_keep_merge_counters.load())
-      MXFA_CUDA(cudaMemsetAsync(sa.sync, 0, sizeof(int) * (size_t)p.batch, st));
+      MXFA_CUDA(cudaMemsetAsync(sa.sync, 0, sizeof(int) * (size_t)n_seq, st));
     void *args[] = {&p, &sa, &mq, &mkv};
-    MXFA_CUDA(cudaLaunchCooperativeKernel(k, dim3(p.batch * sa.arith_k), dim3(threads), args, kDcSmemBytes, st));
+    MXFA_CUDA(cudaLaunchCooperativeKernel(k, dim3(n_seq * sa.arith_k), dim3(threads), args, kDcSmemBytes, st));
     return MXFA_OK;
   }
   decode_prep_kernel<<<1, 1024, 0, st>>>(p, s);
   MXFA_CUDA(cudaGetLastError());
   void *args[] = {&p, &s, &mq, &mkv};
   MXFA_TRY(launch_dependent(k, dim3(s.grid), dim3(threads), kDcSmemBytes, st, args));
-  const int cg = combine_grid(p.batch, kDcDv, s.grid);
-  int ns = p.batch;
+  const int cg = combine_grid(n_seq, kDcDv, s.grid);
+  int ns = n_seq;
   void *cargs[] = {&p, &s, &ns};
   const void *ck = dt == MXFA_BF16 ? reinterpret_cast<const void *>(decode_combine_kernel<__nv_bfloat16, kDcDv>)
                                    : reinterpret_cast<const void *>(decode_combine_kernel<__half, kDcDv>);
@@ -696,10 +712,11 @@ mxfa_status_t mxfa_attn_varlen_fwd(const void *q, const void *k, const void *v, 
 size_t mxfa_attn_decode_splitkv_workspace_size(int batch, int max_q_len, int Hq, int Hkv, int Dv, int max_kv_len,
                                                int num_splits, mxfa_dtype_t dtype) {
   if (dtype == MXFA_F32 || batch <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || num_splits < 0) return sizeof(WsHeader);
-  if (Dv == kDcDv && Hkv == 1 && (int64_t)max_q_len * Hq <= kDcRows)  // MLA
-    return decode_ws(batch, max_kv_len, num_splits, kDcDv, kDcKeys).total;
-  if ((Dv == 64 || Dv == 128) && (int64_t)max_q_len * (Hq / Hkv) <= kDcRows)  // grouped-query heads
-    return decode_ws(batch * Hkv, max_kv_len, num_splits, Dv, kGqKeys).total;
+  const int subs = head_subgroups(Hq / Hkv, max_q_len);
+  if (Dv == kDcDv && Hkv == 1 && subs > 0)  // MLA
+    return decode_ws(batch * subs, max_kv_len, num_splits, kDcDv, kDcKeys).total;
+  if ((Dv == 64 || Dv == 128) && subs > 0)  // grouped-query heads
+    return decode_ws(batch * Hkv * subs, max_kv_len, num_splits, Dv, kGqKeys).total;
   return sizeof(WsHeader);
 }
 
@@ -757,15 +774,17 @@ mxfa_status_t mxfa_attn_decode_splitkv(const void *q, const void *k, const void 
   if (decode_gqa_eligible(dtype, Hq, Hkv, Dqk, Dv, max_q_len, k_row_stride, v_row_stride) && total_kv > 0) {
     int sms = 0;
     MXFA_TRY(sm_count(&sms));
-    const DecodeSched s = decode_sched(p, Hkv, num_splits, Dv, kGqKeys, workspace, sms);
+    const int subs = head_subgroups(Hq / Hkv, max_q_len);
+    const DecodeSched s = decode_sched(p, Hkv * subs, subs, num_splits, Dv, kGqKeys, workspace, sms);
     return launch_decode_gqa(p, s, dtype, total_kv, kGqKeys, st);
   }
   return launch_simt_any(dtype, p, max_q_len, st);
 }
 
 size_t mxfa_attn_decode_mla_fp8kv_workspace_size(int batch, int max_q_len, int Hq, int max_kv_len, int num_splits) {
-  if (batch <= 0 || Hq <= 0 || num_splits < 0 || (int64_t)max_q_len * Hq > kDcRows) return sizeof(WsHeader);
-  return decode_ws(batch, max_kv_len, num_splits, kDcDv, kDcKeys).total;
+  const int subs = Hq > 0 ? head_subgroups(Hq, max_q_len) : 0;
+  if (batch <= 0 || num_splits < 0 || subs == 0) return sizeof(WsHeader);
+  return decode_ws(batch * subs, max_kv_len, num_splits, kDcDv, kDcKeys).total;
 }
 
 mxfa_status_t mxfa_attn_decode_mla_fp8kv(const void *q, const void *kv, float kv_scale, void *o, float *lse,
@@ -778,9 +797,8 @@ mxfa_status_t mxfa_attn_decode_mla_fp8kv(const void *q, const void *kv, float kv
   if (Hq <= 0) return fail(MXFA_ERR_INVALID_ARG, "Hq must be positive (Hq=%d)", Hq);
   if (std::isinf(softmax_scale)) return fail(MXFA_ERR_INVALID_ARG, "softmax_scale is infinite");
   if (!std::isfinite(kv_scale)) return fail(MXFA_ERR_INVALID_ARG, "kv_scale is not finite");
-  if ((int64_t)max_q_len * Hq > kDcRows)
-    return fail(MXFA_ERR_UNSUPPORTED, "max_q_len * Hq = %lld exceeds %d query rows per sequence",
-                (long long)max_q_len * Hq, kDcRows);
+  if (max_q_len > kDcRows)
+    return fail(MXFA_ERR_UNSUPPORTED, "max_q_len = %d exceeds %d queries per sequence", max_q_len, kDcRows);
   if (batch == 0 || total_q == 0) return MXFA_OK;
   if (!qo_indptr || !kv_indptr) return fail(MXFA_ERR_INVALID_ARG, "qo_indptr / kv_indptr is NULL");
   if (max_q_len > total_q || max_kv_len > total_kv)
@@ -817,9 +835,9 @@ mxfa_status_t mxfa_attn_decode_mla_fp8kv(const void *q, const void *kv, float kv
 size_t mxfa_attn_decode_kvcache_workspace_size(int batch, int Sq, int Hq, int Hkv, int D, int max_len,
                                                int num_splits, mxfa_dtype_t dtype) {
   if (dtype == MXFA_F32 || batch <= 0 || Sq <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || num_splits < 0 ||
-      (D != 64 && D != 128) || (int64_t)Sq * (Hq / Hkv) > kDcRows || max_len < 0)
+      (D != 64 && D != 128) || Sq > kDcRows || max_len < 0)
     return sizeof(WsHeader);
-  return decode_ws(batch * Hkv, max_len, num_splits, D, kGqKeys).total;
+  return decode_ws(batch * Hkv * head_subgroups(Hq / Hkv, Sq), max_len, num_splits, D, kGqKeys).total;
 }
 
 mxfa_status_t mxfa_attn_decode_kvcache(const void *q, void *k_cache, void *v_cache, const void *k_new,
@@ -836,9 +854,7 @@ mxfa_status_t mxfa_attn_decode_kvcache(const void *q, void *k_cache, void *v_cac
   if (D != 64 && D != 128) return fail(MXFA_ERR_UNSUPPORTED, "head dimension %d is not 64 or 128", D);
   if (std::isinf(softmax_scale)) return fail(MXFA_ERR_INVALID_ARG, "softmax_scale is infinite");
   if (dtype == MXFA_F32) return fail(MXFA_ERR_UNSUPPORTED, "the KV-cache decode takes bf16 or f16");
-  if ((int64_t)Sq * (Hq / Hkv) > kDcRows)
-    return fail(MXFA_ERR_UNSUPPORTED, "Sq * Hq / Hkv = %lld query rows per KV head exceed %d",
-                (long long)Sq * (Hq / Hkv), kDcRows);
+  if (Sq > kDcRows) return fail(MXFA_ERR_UNSUPPORTED, "Sq = %d exceeds %d queries per sequence", Sq, kDcRows);
   if ((k_new == nullptr) != (v_new == nullptr) || (Snew > 0 && k_new == nullptr))
     return fail(MXFA_ERR_INVALID_ARG, "k_new and v_new go together, and Snew > 0 needs them");
   if (batch == 0 || Sq == 0) return MXFA_OK;
@@ -881,7 +897,8 @@ mxfa_status_t mxfa_attn_decode_kvcache(const void *q, void *k_cache, void *v_cac
   p.wait_ns = g_wait_ns.load();
   int sms = 0;
   MXFA_TRY(sm_count(&sms));
-  DecodeSched s = decode_sched(p, Hkv, num_splits, D, kGqKeys, workspace, sms);
+  const int subs = head_subgroups(Hq / Hkv, Sq);
+  DecodeSched s = decode_sched(p, Hkv * subs, subs, num_splits, D, kGqKeys, workspace, sms);
   s.cache_seqlens = cache_seqlens;
   s.add = Snew;
   s.advance = Snew > 0 ? 1 : 0;
