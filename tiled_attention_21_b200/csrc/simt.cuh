@@ -23,13 +23,14 @@ namespace mxfa {
 
 constexpr int kSimtWarps = 8;
 constexpr int kSimtKeys = 32;
+constexpr int kSimtStage = 8;  // loads in flight per thread while a tile is staged
 
 __host__ __device__ inline size_t simt_smem_bytes(int dqk, int dv) {
   return sizeof(float) * ((size_t)kSimtWarps * dqk + (size_t)kSimtKeys * (dqk + 1) + (size_t)kSimtKeys * dv);
 }
 
 template <typename T, int DV_PER_LANE>
-__global__ void __launch_bounds__(kSimtWarps * 32)
+__global__ void __launch_bounds__(kSimtWarps * 32, 2)
 attn_fwd_simt_kernel(const AttnParams p) {
   extern __shared__ float smem[];
   const int dqk = p.dqk, dv = p.dv;
@@ -68,13 +69,34 @@ attn_fwd_simt_kernel(const AttnParams p) {
   for (int t0 = 0; t0 < block_keys; t0 += kSimtKeys) {
     __syncthreads();  // previous tile fully consumed (also orders the qs writes)
     const int nk = min(kSimtKeys, block_keys - t0);
-    for (int idx = threadIdx.x; idx < kSimtKeys * dqk; idx += blockDim.x) {
-      int j = idx / dqk, d = idx - j * dqk;
-      ks[j * (dqk + 1) + d] = j < nk ? to_f32(kbase[(int64_t)(sr.k0 + t0 + j) * p.k_rs + d]) : 0.f;
-    }
-    for (int idx = threadIdx.x; idx < kSimtKeys * dv; idx += blockDim.x) {
-      int j = idx / dv, d = idx - j * dv;
-      vs[j * dv + d] = j < nk ? to_f32(vbase[(int64_t)(sr.k0 + t0 + j) * p.v_rs + d]) : 0.f;
+    // Stage the K and V tiles: each thread issues a batch of independent
+    // loads before it stores any of them, so a tile costs about one memory
+    // latency rather than one per element.
+    for (int base = threadIdx.x; base < kSimtKeys * (dqk + dv); base += kSimtStage * kSimtWarps * 32) {
+      float x[kSimtStage];
+#pragma unroll
+      for (int u = 0; u < kSimtStage; ++u) {
+        const int idx = base + u * kSimtWarps * 32;
+        x[u] = 0.f;
+        if (idx < kSimtKeys * dqk) {
+          const int j = idx / dqk, d = idx - j * dqk;
+          if (j < nk) x[u] = to_f32(kbase[(int64_t)(sr.k0 + t0 + j) * p.k_rs + d]);
+        } else if (idx < kSimtKeys * (dqk + dv)) {
+          const int jv = idx - kSimtKeys * dqk, j = jv / dv, d = jv - j * dv;
+          if (j < nk) x[u] = to_f32(vbase[(int64_t)(sr.k0 + t0 + j) * p.v_rs + d]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kSimtStage; ++u) {
+        const int idx = base + u * kSimtWarps * 32;
+        if (idx < kSimtKeys * dqk) {
+          const int j = idx / dqk, d = idx - j * dqk;
+          ks[j * (dqk + 1) + d] = x[u];
+        } else if (idx < kSimtKeys * (dqk + dv)) {
+          const int jv = idx - kSimtKeys * dqk, j = jv / dv, d = jv - j * dv;
+          vs[j * dv + d] = x[u];
+        }
+      }
     }
     __syncthreads();
     if (!active || t0 >= n_vis) continue;
