@@ -330,7 +330,9 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": headline_config(p, flops, world) | {"l2": "n/a (host)"},
+            "config": headline_config(p, flops, world),
+            "host_note": "the oracle runs on the host cores on sampled rows of this workload; "
+                         "the config's L2 policy is the GPU arm's",
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

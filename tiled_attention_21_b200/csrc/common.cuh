@@ -55,6 +55,7 @@ struct AttnParams {
   WsHeader *hdr;
   const int2 *pairs;          // varlen schedule: sorted (sequence, 256-row block) pairs
   uint64_t wait_ns;           // budget of every bounded device-side wait (kWaitBudgetNs unless a test shortens it)
+  int paired;                 // tensor-core prefill: deal units as pairs of 256-row blocks (see unit_at)
 };
 
 struct SeqRange {

@@ -275,10 +275,16 @@ mxfa_status_t launch_simt_any(mxfa_dtype_t dt, const AttnParams &p, int max_rows
 }
 
 template <int D, bool BF16>
-mxfa_status_t launch_tc(const AttnParams &p, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+mxfa_status_t launch_tc(AttnParams &p, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                         cudaStream_t st) {
   int sms = 0;
   MXFA_TRY(sm_count(&sms));
+  // Long causal sequences of one length: units dealt as equal-cost pairs of
+  // blocks, heads together (L2 reuse of K/V), when there are at least eight
+  // pairs per CTA, so the coarser items still balance.
+  const int64_t nblk = ((int64_t)p.sq + kTcUnitRows - 1) / kTcUnitRows;
+  p.paired = (p.cu_q == nullptr && p.causal && p.sq == p.sk && nblk % 2 == 0 &&
+              (int64_t)p.batch * p.hq * (nblk / 2) >= 8 * (int64_t)sms) ? 1 : 0;
   auto k = attn_fwd_tc_kernel<D, BF16>;
   if (kTcRegsIo != kTcLaunchRegs || kTcRegsSoftmax != kTcLaunchRegs)  // a setmaxnreg split is compiled in
     MXFA_TRY(check_launch_regs(reinterpret_cast<const void *>(k), kTcLaunchRegs));

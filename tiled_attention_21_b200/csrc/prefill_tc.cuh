@@ -104,24 +104,9 @@ struct UnitInfo {
   int n[2];  // KV tiles needed by query tile 0 / 1
 };
 
-// Unit u of the schedule.  Uniform lengths: 256-row blocks ordered by
-// decreasing causal cost (last block first), all sequences of a block
-// consecutively, heads innermost.  Varlen: the (b, m) pairs sorted by the
-// prep kernel.
-__device__ __forceinline__ UnitInfo unit_info(const AttnParams &p, int u) {
-  UnitInfo ui;
-  const int pr = u / p.hq;
-  ui.h = u - pr * p.hq;
+// The work of unit (b, m, h): its KV-tile counts per query tile.
+__device__ __forceinline__ void unit_fill(const AttnParams &p, UnitInfo &ui) {
   ui.g = ui.h / (p.hq / p.hkv);
-  if (p.cu_q == nullptr) {
-    const int nblk = (p.sq + kTcUnitRows - 1) / kTcUnitRows;
-    ui.m = nblk - 1 - pr / p.batch;
-    ui.b = pr - (pr / p.batch) * p.batch;
-  } else {
-    const int2 pm = p.pairs[pr];
-    ui.b = pm.x;
-    ui.m = pm.y;
-  }
   ui.sr = seq_range(p, ui.b);
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
@@ -133,6 +118,26 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams &p, int u) {
       ui.n[t] = (visible_keys(last, ui.sr.sq, ui.sr.sk, p.causal) + kTcBlockN - 1) / kTcBlockN;
     }
   }
+}
+
+// Unit u of the schedule.  Uniform lengths: 256-row blocks ordered by
+// decreasing causal cost (last block first), all sequences of a block
+// consecutively, heads innermost.  Varlen: the (b, m) pairs sorted by the
+// prep kernel.
+__device__ __forceinline__ UnitInfo unit_info(const AttnParams &p, int u) {
+  UnitInfo ui;
+  const int pr = u / p.hq;
+  ui.h = u - pr * p.hq;
+  if (p.cu_q == nullptr) {
+    const int nblk = (p.sq + kTcUnitRows - 1) / kTcUnitRows;
+    ui.m = nblk - 1 - pr / p.batch;
+    ui.b = pr - (pr / p.batch) * p.batch;
+  } else {
+    const int2 pm = p.pairs[pr];
+    ui.b = pm.x;
+    ui.m = pm.y;
+  }
+  unit_fill(p, ui);
   return ui;
 }
 
@@ -145,6 +150,34 @@ __device__ __forceinline__ int unit_of(int round, int cta, int grid) {
 __device__ __forceinline__ int n_units_of(const AttnParams &p) {
   if (p.cu_q == nullptr) return p.batch * ((p.sq + kTcUnitRows - 1) / kTcUnitRows) * p.hq;
   return (int)(*reinterpret_cast<volatile uint32_t *>(&p.hdr->n_units)) * p.hq;
+}
+
+// The unit of this CTA's iteration `it` (false once the CTA has no more).
+// Default: unit unit_of(it) of the list above (heaviest first, so the
+// persistent CTAs finish close together).  Paired (p.paired, long causal
+// sequences of uniform length with an even number of 256-row blocks): a work
+// item is block nblk-1-k followed by block k of one (sequence, head), whose
+// causal costs add up to the same number of KV tiles for every k; the items
+// are dealt in the snake order with the k of one (sequence, head)
+// consecutive, so the CTAs running at any time cover about 148 / (nblk/2)
+// heads and their K/V streams share L2 instead of each head's K/V being
+// re-read from DRAM by every block of it.
+__device__ __forceinline__ bool unit_at(const AttnParams &p, int it, int cta, int grid, int n_units, UnitInfo &ui) {
+  if (!p.paired) {
+    const int u = unit_of(it, cta, grid);
+    if (u >= n_units) return false;
+    ui = unit_info(p, u);
+    return true;
+  }
+  const int npairs = (p.sq + kTcUnitRows - 1) / kTcUnitRows / 2;
+  const int item = unit_of(it >> 1, cta, grid);
+  if (item >= n_units / 2) return false;
+  const int bh = item / npairs, k = item - bh * npairs;
+  ui.b = bh / p.hq;
+  ui.h = bh - ui.b * p.hq;
+  ui.m = (it & 1) ? k : 2 * npairs - 1 - k;
+  unit_fill(p, ui);
+  return true;
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -328,8 +361,8 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     if (lane == 0) {
       uint32_t ring = 0, q_issued = 0;
       bool ok = true;
-      for (int it = 0, u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
-        const UnitInfo ui = unit_info(p, u);
+      UnitInfo ui;
+      for (int it = 0; ok && unit_at(p, it, cta, grid, n_units, ui); ++it) {
         const int nmax = max(ui.n[0], ui.n[1]);
         if (it > 0 && !wait_bar(b_qe, (it - 1) & 1, abort_flag, hdr, kSiteQEmpty, p.wait_ns)) break;
         mbar_arrive_expect_tx(b_qf, 2 * Cfg::kTileBytes);
@@ -411,8 +444,8 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       };
       int it = 0;
       bool ok = true;
-      for (int u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
-        const UnitInfo ui = unit_info(p, u);
+      UnitInfo ui;
+      for (; ok && unit_at(p, it, cta, grid, n_units, ui); ++it) {
         const int nmax = max(ui.n[0], ui.n[1]);
         if (!wait_warp(b_qf, it & 1, abort_flag, hdr, kSiteQFull)) break;
         tc_fence_after();
@@ -508,8 +541,8 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     uint32_t s_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
     int it = 0;
     bool ok = true;
-    for (int u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
-      const UnitInfo ui = unit_info(p, u);
+    UnitInfo ui;
+    for (; ok && unit_at(p, it, cta, grid, n_units, ui); ++it) {
       const int nmax = max(ui.n[0], ui.n[1]);
       int i[2], nv[2];
       float m_used[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
@@ -635,8 +668,8 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
     uint32_t o_cnt[2] = {0, 0};
     bool ok = true;
-    for (int it = 0, u; ok && (u = unit_of(it, cta, grid)) < n_units; ++it) {
-      const UnitInfo ui = unit_info(p, u);
+    UnitInfo ui;
+    for (int it = 0; ok && unit_at(p, it, cta, grid, n_units, ui); ++it) {
       const bool got_l = wait_bar(smem_u32(&ctrl->l_ready), it & 1, abort_flag, hdr, kSiteLReady, p.wait_ns);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got_l)) break;

@@ -59,9 +59,9 @@ attn_fwd_simt_kernel(const AttnParams p) {
   for (int d = lane; d < dqk; d += 32) qs[warp * dqk + d] = active ? to_f32(qrow[d]) : 0.f;
 
   float m = -INFINITY, l = 0.f;
-  float acc[DV_PER_LANE];
+  float acc[DV_PER_LANE], acc2[DV_PER_LANE];
 #pragma unroll
-  for (int e = 0; e < DV_PER_LANE; ++e) acc[e] = 0.f;
+  for (int e = 0; e < DV_PER_LANE; ++e) acc[e] = acc2[e] = 0.f;
 
   const T *kbase = reinterpret_cast<const T *>(p.k) + (int64_t)g * p.k_hs;
   const T *vbase = reinterpret_cast<const T *>(p.v) + (int64_t)g * p.v_hs;
@@ -101,11 +101,16 @@ attn_fwd_simt_kernel(const AttnParams p) {
     __syncthreads();
     if (!active || t0 >= n_vis) continue;
 
-    // score of key t0 + lane, in the log2 domain
-    float s = 0.f;
+    // score of key t0 + lane, in the log2 domain: four partial sums over
+    // d mod 4 (dqk is a multiple of 4), so the FMA chain is a quarter as long
     const float *kr = ks + lane * (dqk + 1);
     const float *qr = qs + warp * dqk;
-    for (int d = 0; d < dqk; ++d) s = fmaf(qr[d], kr[d], s);
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int d = 0; d < dqk; d += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) s4[u] = fmaf(qr[d + u], kr[d + u], s4[u]);
+    }
+    const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
     float x = (t0 + lane < n_vis) ? s * p.scale_log2 : -INFINITY;
 
     float tmax = x;
@@ -122,13 +127,20 @@ attn_fwd_simt_kernel(const AttnParams p) {
     m = m_new;
 #pragma unroll
     for (int e = 0; e < DV_PER_LANE; ++e) acc[e] *= alpha;
-    for (int j = 0; j < nk; ++j) {
-      const float pb = __shfl_sync(0xffffffffu, pj, j);
-      const float *vr = vs + j * dv;
+#pragma unroll
+    for (int e = 0; e < DV_PER_LANE; ++e) acc2[e] *= alpha;
+    // P.V: even and odd keys accumulate separately (two independent chains;
+    // keys past nk have pj = 0 and zero-filled V rows)
+    for (int j = 0; j < nk; j += 2) {
+      const float pa = __shfl_sync(0xffffffffu, pj, j), pb = __shfl_sync(0xffffffffu, pj, j + 1);
+      const float *va = vs + j * dv, *vb = va + dv;
 #pragma unroll
       for (int e = 0; e < DV_PER_LANE; ++e) {
         const int d = lane + 32 * e;
-        if (d < dv) acc[e] = fmaf(pb, vr[d], acc[e]);
+        if (d < dv) {
+          acc[e] = fmaf(pa, va[d], acc[e]);
+          acc2[e] = fmaf(pb, vb[d], acc2[e]);
+        }
       }
     }
   }
@@ -139,7 +151,7 @@ attn_fwd_simt_kernel(const AttnParams p) {
 #pragma unroll
   for (int e = 0; e < DV_PER_LANE; ++e) {
     const int d = lane + 32 * e;
-    if (d < dv) orow[d] = from_f32<T>(acc[e] * inv);
+    if (d < dv) orow[d] = from_f32<T>((acc[e] + acc2[e]) * inv);
   }
   if (p.lse && lane == 0) {
     const float lse = l > 0.f ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
