@@ -198,3 +198,12 @@ def test_varlen_max_seqlen_below_a_length_is_reported():
     assert mx.read_device_status(ws)[0] == mx.MXFA_OK
     ro, rl = oracle.problem(p)
     compare(o, l, ro, rl, p.q.dtype, p.name)
+
+
+def test_varlen_many_heads_sampled():
+    """A causal varlen problem with 64 query heads over 8 KV heads, odd and
+    even 256-row block counts, and a one-row and a 255-row sequence, checked
+    on sampled rows including every sequence's first and last row."""
+    p = workloads.varlen(21, [3000, 2500, 2131, 1900, 255, 1], [3000, 2500, 2131, 1900, 255, 1], 64, 8, 128,
+                         "bf16", True)
+    _sampled(p, 6, 104)

@@ -25,6 +25,7 @@ constexpr int kSimtWarps = 8;
 constexpr int kSimtKeys = 32;
 constexpr int kSimtStage = 8;  // loads in flight per thread while a tile is staged
 
+
 __host__ __device__ inline size_t simt_smem_bytes(int dqk, int dv) {
   return sizeof(float) * ((size_t)kSimtWarps * dqk + (size_t)kSimtKeys * (dqk + 1) + (size_t)kSimtKeys * dv);
 }
@@ -66,37 +67,53 @@ attn_fwd_simt_kernel(const AttnParams p) {
   const T *kbase = reinterpret_cast<const T *>(p.k) + (int64_t)g * p.k_hs;
   const T *vbase = reinterpret_cast<const T *>(p.v) + (int64_t)g * p.v_hs;
 
+  // K and V tiles are staged in 16-byte pieces: a thread issues a batch of
+  // independent loads before it converts and stores any of them, so a tile
+  // costs about one memory latency.  Rows are 16-byte aligned (the entry
+  // points check the pointers and strides), and dqk, dv are multiples of the
+  // eight or four elements of a piece.
+  constexpr int kVec = 16 / sizeof(T);
+  constexpr int kBatch = kSimtStage * kSimtWarps * 32;
+  const int kq = dqk / kVec, vq = dv / kVec;
+  const int n_pieces = kSimtKeys * (kq + vq);
+  auto load = [&](int t, int base, uint4 (&w)[kSimtStage]) {
+    const int nk = min(kSimtKeys, block_keys - t);
+#pragma unroll
+    for (int u = 0; u < kSimtStage; ++u) {
+      const int c = base + u * kSimtWarps * 32;
+      w[u] = make_uint4(0, 0, 0, 0);
+      if (c < kSimtKeys * kq) {
+        const int j = c / kq, dc = c - j * kq;
+        if (j < nk) w[u] = *reinterpret_cast<const uint4 *>(kbase + (int64_t)(sr.k0 + t + j) * p.k_rs + dc * kVec);
+      } else if (c < n_pieces) {
+        const int cv = c - kSimtKeys * kq, j = cv / vq, dc = cv - j * vq;
+        if (j < nk) w[u] = *reinterpret_cast<const uint4 *>(vbase + (int64_t)(sr.k0 + t + j) * p.v_rs + dc * kVec);
+      }
+    }
+  };
+  auto store = [&](int base, const uint4 (&w)[kSimtStage]) {
+#pragma unroll
+    for (int u = 0; u < kSimtStage; ++u) {
+      const int c = base + u * kSimtWarps * 32;
+      const T *e = reinterpret_cast<const T *>(&w[u]);
+      if (c < kSimtKeys * kq) {
+        const int j = c / kq, dc = c - j * kq;
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) ks[j * (dqk + 1) + dc * kVec + i] = to_f32(e[i]);
+      } else if (c < n_pieces) {
+        const int cv = c - kSimtKeys * kq, j = cv / vq, dc = cv - j * vq;
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) vs[j * dv + dc * kVec + i] = to_f32(e[i]);
+      }
+    }
+  };
   for (int t0 = 0; t0 < block_keys; t0 += kSimtKeys) {
     __syncthreads();  // previous tile fully consumed (also orders the qs writes)
     const int nk = min(kSimtKeys, block_keys - t0);
-    // Stage the K and V tiles: each thread issues a batch of independent
-    // loads before it stores any of them, so a tile costs about one memory
-    // latency rather than one per element.
-    for (int base = threadIdx.x; base < kSimtKeys * (dqk + dv); base += kSimtStage * kSimtWarps * 32) {
-      float x[kSimtStage];
-#pragma unroll
-      for (int u = 0; u < kSimtStage; ++u) {
-        const int idx = base + u * kSimtWarps * 32;
-        x[u] = 0.f;
-        if (idx < kSimtKeys * dqk) {
-          const int j = idx / dqk, d = idx - j * dqk;
-          if (j < nk) x[u] = to_f32(kbase[(int64_t)(sr.k0 + t0 + j) * p.k_rs + d]);
-        } else if (idx < kSimtKeys * (dqk + dv)) {
-          const int jv = idx - kSimtKeys * dqk, j = jv / dv, d = jv - j * dv;
-          if (j < nk) x[u] = to_f32(vbase[(int64_t)(sr.k0 + t0 + j) * p.v_rs + d]);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kSimtStage; ++u) {
-        const int idx = base + u * kSimtWarps * 32;
-        if (idx < kSimtKeys * dqk) {
-          const int j = idx / dqk, d = idx - j * dqk;
-          ks[j * (dqk + 1) + d] = x[u];
-        } else if (idx < kSimtKeys * (dqk + dv)) {
-          const int jv = idx - kSimtKeys * dqk, j = jv / dv, d = jv - j * dv;
-          vs[j * dv + d] = x[u];
-        }
-      }
+    for (int base = threadIdx.x; base < n_pieces; base += kBatch) {
+      uint4 w[kSimtStage];
+      load(t0, base, w);
+      store(base, w);
     }
     __syncthreads();
     if (!active || t0 >= n_vis) continue;
