@@ -82,3 +82,10 @@ def test_graph_mla_decode_fp8kv():
     b = workloads.mla_decode_fp8(60, batch=4, q_len=4, kv_len=1024)
     b.kv_scale = a.kv_scale  # the scale is a call argument, captured with the graph
     _replay_matches(a, b, "decode")
+
+
+def test_graph_mla_decode_head_groups():
+    # 8 queries x 16 heads: two head groups, three kernels (more sequences than one launch takes)
+    a = workloads.mla_decode(61, batch=96, q_len=8, kv_len=1500)
+    b = workloads.mla_decode(62, batch=96, q_len=8, kv_len=1500)
+    _replay_matches(a, b, "decode")
