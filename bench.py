@@ -321,8 +321,8 @@ def run_reference(args, rank, world):
         return
     p = headline_problem()
     flops = prefill_flops(HEADLINE["B"], HEADLINE["H"], HEADLINE["S"], HEADLINE["D"])
-    res = [cpu_baseline(p, "flops", target_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
-           for _ in range(args.warmup + args.steps)]
+    per_step = args.sample_seconds if args.sample_seconds else max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    res = [cpu_baseline(p, "flops", target_s=per_step) for _ in range(args.warmup + args.steps)]
     vals = [r["value"] for r in res[args.warmup:]]
     v = statistics.mean(vals)
     cb = dict(res[-1])
@@ -600,6 +600,8 @@ def main():
                     choices=["headline", "batched_causal", "varlen_gqa", "single_head_fp32", "decode", "mla_q8", "gqa",
                              "fp8"],
                     help="time one workload only (used for profiling captures; no JSON contract line)")
+    ap.add_argument("--sample-seconds", type=float, default=None,
+                    help="reference arm: seconds of oracle work per step (default: about a minute in all)")
     ap.add_argument("--decode-batch", type=int, default=128,
                     help="sequences of the MLA decode workloads (128 = the full workload; smaller for captures)")
     args = ap.parse_args()

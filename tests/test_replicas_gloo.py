@@ -78,3 +78,25 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
 
     b.run_reference(Args, 1, 2)                        # rank 1: no work, no output
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores, on
+    sampled rows of the headline workload) prints one JSON line with the
+    contract's keys and the headline's config."""
+    import json
+    import subprocess
+    import sys as _sys
+    out = subprocess.run([_sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "3", "--sample-seconds", "0.3"], capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "higher_is_better", "scaling", "dtype",
+                "data", "config", "cpu_baseline", "e2e", "impl"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    b = _bench()
+    assert d["config"] == b.headline_config_of(d["config"]["workload"], d["config"]["flops_per_step"], 1)
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
