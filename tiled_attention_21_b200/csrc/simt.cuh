@@ -76,6 +76,9 @@ attn_fwd_simt_kernel(const AttnParams p) {
   constexpr int kBatch = kSimtStage * kSimtWarps * 32;
   const int kq = dqk / kVec, vq = dv / kVec;
   const int n_pieces = kSimtKeys * (kq + vq);
+  // c / kq and c / vq as a multiply-high by ceil(2^32 / divisor): exact for
+  // c * divisor^2 < 2^32 (here c < 32 * 288 and divisors <= 144)
+  const uint32_t mk = (uint32_t)(((1ull << 32) + kq - 1) / kq), mv = (uint32_t)(((1ull << 32) + vq - 1) / vq);
   auto load = [&](int t, int base, uint4 (&w)[kSimtStage]) {
     const int nk = min(kSimtKeys, block_keys - t);
 #pragma unroll
@@ -83,10 +86,10 @@ attn_fwd_simt_kernel(const AttnParams p) {
       const int c = base + u * kSimtWarps * 32;
       w[u] = make_uint4(0, 0, 0, 0);
       if (c < kSimtKeys * kq) {
-        const int j = c / kq, dc = c - j * kq;
+        const int j = (int)__umulhi((uint32_t)c, mk), dc = c - j * kq;
         if (j < nk) w[u] = *reinterpret_cast<const uint4 *>(kbase + (int64_t)(sr.k0 + t + j) * p.k_rs + dc * kVec);
       } else if (c < n_pieces) {
-        const int cv = c - kSimtKeys * kq, j = cv / vq, dc = cv - j * vq;
+        const int cv = c - kSimtKeys * kq, j = (int)__umulhi((uint32_t)cv, mv), dc = cv - j * vq;
         if (j < nk) w[u] = *reinterpret_cast<const uint4 *>(vbase + (int64_t)(sr.k0 + t + j) * p.v_rs + dc * kVec);
       }
     }
@@ -97,11 +100,11 @@ attn_fwd_simt_kernel(const AttnParams p) {
       const int c = base + u * kSimtWarps * 32;
       const T *e = reinterpret_cast<const T *>(&w[u]);
       if (c < kSimtKeys * kq) {
-        const int j = c / kq, dc = c - j * kq;
+        const int j = (int)__umulhi((uint32_t)c, mk), dc = c - j * kq;
 #pragma unroll
         for (int i = 0; i < kVec; ++i) ks[j * (dqk + 1) + dc * kVec + i] = to_f32(e[i]);
       } else if (c < n_pieces) {
-        const int cv = c - kSimtKeys * kq, j = cv / vq, dc = cv - j * vq;
+        const int cv = c - kSimtKeys * kq, j = (int)__umulhi((uint32_t)cv, mv), dc = cv - j * vq;
 #pragma unroll
         for (int i = 0; i < kVec; ++i) vs[j * dv + dc * kVec + i] = to_f32(e[i]);
       }
