@@ -37,6 +37,15 @@ __device__ __forceinline__ uint64_t global_ns() {
 __device__ __forceinline__ void report_error(WsHeader *hdr, uint32_t code, uint32_t site) {
   if (atomicCAS(&hdr->status, 0u, code) == 0u) atomicExch(&hdr->detail, site);
 }
+// The same, out of line, for the kernels without a setmaxnreg register split
+// (the decode kernels): it runs only when a wait gives up or a schedule
+// overflows, and inlined at every bounded wait it made their hot loops longer
+// (twice the instruction-cache misses in the grouped-query decode, 4 % of its
+// time).  The prefill kernel keeps the inline form, so no call is made from
+// a warp whose register budget setmaxnreg has lowered.
+__device__ __noinline__ void report_error_cold(WsHeader *hdr, uint32_t code, uint32_t site) {
+  report_error(hdr, code, site);
+}
 
 // Common parameter block of the attention kernels.  Lengths are either
 // uniform (cu_q == nullptr: sequence b holds tokens [b*sq, (b+1)*sq)) or

@@ -131,7 +131,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
         const int len = dc_klen(p, s, b);
         for (int j = sd.y; ok && j < sd.z; ++j, ++tc) {
           const int x = tc % Cfg::kRingTiles;
-          if (!wait_bar(b_te(x), ((tc / Cfg::kRingTiles) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty, p.wait_ns)) {
+          if (!wait_bar<kDcColdReport>(b_te(x), ((tc / Cfg::kRingTiles) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -168,7 +168,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
     // lane issues each tcgen05 operation; the warp gives up a wait together.
     const bool leader = elect_one();
     auto wait_warp = [&](uint32_t bar, uint32_t parity, uint32_t site) {
-      return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, hdr, site, p.wait_ns));
+      return __all_sync(0xffffffffu, wait_bar<kDcColdReport>(bar, parity, abort_flag, hdr, site, p.wait_ns));
     };
     constexpr uint32_t idesc_s = make_idesc_f16(BF16, kDcRows, kGqKeys, false, false);
     constexpr uint32_t idesc_o = make_idesc_f16(BF16, kDcRows, D, false, true);
@@ -284,7 +284,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
       const int nv = valid ? visible_keys(r / G, sq, sk, p.causal) : 0;
       float m_used = -INFINITY, l = 0.f;
       for (int j = sd.y; j < sd.z; ++j, ++g) {
-        const bool got = wait_bar(b_sf, g & 1, abort_flag, hdr, kDSiteSFull, p.wait_ns);
+        const bool got = wait_bar<kDcColdReport>(b_sf, g & 1, abort_flag, hdr, kDSiteSFull, p.wait_ns);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
@@ -343,7 +343,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
         l = l * alpha + rs;
         // P (single buffer) and O may be touched only once the previous P.V is done.
         if (g > 0) {
-          const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
+          const bool got_o = wait_bar<kDcColdReport>(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got_o)) {
             ok = false;
@@ -384,7 +384,7 @@ attn_decode_gqa_kernel(const __grid_constant__ AttnParams p, const DecodeSched s
       // ---------------- epilogue of this piece
       l += __shfl_xor_sync(0xffffffffu, l, 16);
       if (sd.z > sd.y) {
-        const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
+        const bool got_o = wait_bar<kDcColdReport>(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got_o)) break;
         tc_fence_after();
@@ -465,7 +465,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AttnParams p, cons
     row = page >= 0 ? page * s.page_size + pos % s.page_size : -1;
   }
   if (row < 0 || row >= num_rows) {
-    if (threadIdx.x == 0) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x501);
+    if (threadIdx.x == 0) report_error_cold(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x501);
     return;
   }
   const int per_row = p.hkv * p.dqk / 8;  // 16-byte pieces of one token's K (or V)

@@ -57,6 +57,8 @@ constexpr int kDcCtrlBytes = 2048;
 constexpr int kDcSmemBytes = kDcCtrlBytes + kDcSlots * kDcChunkBytes + kDcRows * 128;
 static_assert(kDcSmemBytes <= 232448, "shared memory budget");
 constexpr int kDcMaxGrid = 256;
+// The decode kernels have no register split: their error reports are calls.
+constexpr bool kDcColdReport = true;
 
 // A decode "sequence" v is (batch entry b, head group gh) (dc_seq): the
 // G = Hq/heads query heads gh*G .. gh*G+G-1 of b, which read KV head
@@ -68,6 +70,16 @@ constexpr int kDcMaxGrid = 256;
 // entries of group 0, then of group 1, ...), so the groups of one batch
 // entry land on CTAs far apart in the tile order and read the same tiles at
 // about the same time, the later reads from L2.
+// n / d for 0 <= n < 2^31 as (n * m) >> sh with sh = 31 + ceil(log2 d) and
+// m = ceil(2^sh / d) (the round-up method of division by invariant integers,
+// Granlund and Montgomery 1994): exact because n * (m * d - 2^sh) < 2^31 * d
+// <= 2^sh.  A multiply and a shift in place of a division sequence.
+struct DivU {
+  uint32_t m, sh;
+  int d;
+};
+__device__ __forceinline__ int div_u(int n, const DivU &q) { return (int)(((uint64_t)(uint32_t)n * q.m) >> q.sh); }
+
 struct DecodeSched {
   int heads;       // head groups per batch entry that form separate sequences
   int subs;        // head groups per KV head
@@ -111,6 +123,7 @@ struct DecodeSched {
   // dequantisation scale of the fp8-KV MLA kernel (the scores' share of that
   // scale is folded into AttnParams::scale_log2 by the host).
   float o_scale;
+  DivU by_bh, by_hkv;  // divisors of dc_seq: batch * Hkv and Hkv
 };
 
 struct DcSeq {
@@ -118,12 +131,10 @@ struct DcSeq {
 };
 // v = (sub * batch + b) * Hkv + kvh with gh = kvh * subs + sub.
 __device__ __forceinline__ DcSeq dc_seq(const AttnParams &p, const DecodeSched &s, int v) {
-  const int hkv = s.heads / s.subs;
-  const int n_bh = p.batch * hkv;
-  const int sub = v / n_bh, w = v - sub * n_bh;
+  const int sub = div_u(v, s.by_bh), w = v - sub * s.by_bh.d;
   DcSeq r;
-  r.b = w / hkv;
-  r.kvh = w - r.b * hkv;
+  r.b = div_u(w, s.by_hkv);
+  r.kvh = w - r.b * s.by_hkv.d;
   r.gh = r.kvh * s.subs + sub;
   return r;
 }
@@ -265,7 +276,7 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
         // no page at all, so the length is cut there and the call reports it.
         const int64_t cap = s.block_table ? (int64_t)s.max_blocks * s.page_size : (int64_t)s.page_size;
         if (len > cap) {
-          if (sq_b.gh == 0) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x402);
+          if (sq_b.gh == 0) report_error_cold(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x402);
           len = (int)cap;
         }
         if (sq_b.gh == 0) s.kv_len[e] = len;
@@ -386,7 +397,7 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     p.hdr->n_units = (uint32_t)min(n_segs, s.max_segs);
     p.hdr->n_aux = (uint32_t)T;
     *s.n_multi = n_multi;
-    if (n_segs > s.max_segs) report_error(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x401);
+    if (n_segs > s.max_segs) report_error_cold(p.hdr, 1u /* MXFA_ERR_INVALID_ARG */, 0x401);
   }
 }
 
@@ -417,7 +428,7 @@ __device__ void dc_merge_pieces(const AttnParams &p, const DecodeSched &s, int v
     int good = 1;
     while (*reinterpret_cast<volatile int *>(s.sync + v) < k) {
       if (global_ns() - t0 > p.wait_ns) {
-        report_error(p.hdr, kStatusTimeout, kDSiteMerge);
+        report_error_cold(p.hdr, kStatusTimeout, kDSiteMerge);
         good = 0;
         break;
       }
@@ -644,7 +655,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         }
         for (int j = sd.y; ok && j < sd.z; ++j, ++tc) {
           const int x = tc % RT;
-          if (!wait_bar(b_te(x), ((tc / RT) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty, p.wait_ns)) {
+          if (!wait_bar<kDcColdReport>(b_te(x), ((tc / RT) & 1) ^ 1, abort_flag, hdr, kDSiteSlotEmpty, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -684,7 +695,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
     // the warp gives up a wait together if any lane gave up.
     const bool leader = elect_one();
     auto wait_warp = [&](uint32_t bar, uint32_t parity, volatile int *ab, WsHeader *h, uint32_t site) {
-      return __all_sync(0xffffffffu, wait_bar(bar, parity, ab, h, site, p.wait_ns));
+      return __all_sync(0xffffffffu, wait_bar<kDcColdReport>(bar, parity, ab, h, site, p.wait_ns));
     };
     {
       constexpr uint32_t idesc_s = make_idesc_f16(BF16, kDcRows, kDcKeys, false, false);
@@ -818,7 +829,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       const int4 sd = dc_seg(p, s, sg);
       for (int j = sd.y; j < sd.z; ++j, ++tc) {
         const int y = tc % RT;
-        if (!agree(wait_bar(b_gf(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull, p.wait_ns))) {
+        if (!agree(wait_bar<kDcColdReport>(b_gf(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -831,7 +842,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         mbar_arrive(b_lf(y));  // S may start on chunks 0-2
         // chunks 3-8 (from chunk 4 on) overwrite codes: every thread reads
         // its groups (and has read its chunk 0-2 groups) before any write
-        if (!agree(wait_bar(b_gr(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull, p.wait_ns))) {
+        if (!agree(wait_bar<kDcColdReport>(b_gr(y), (tc / RT) & 1, abort_flag, hdr, kDSiteStageFull, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -905,7 +916,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       const int nv = valid ? visible_keys(r / G, sq, sk, p.causal) : 0;
       float m_used = -INFINITY, l = 0.f;
       for (int j = sd.y; j < sd.z; ++j, ++g) {
-        const bool got = wait_bar(b_sf, g & 1, abort_flag, hdr, kDSiteSFull, p.wait_ns);
+        const bool got = wait_bar<kDcColdReport>(b_sf, g & 1, abort_flag, hdr, kDSiteSFull, p.wait_ns);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
@@ -956,7 +967,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
         l = l * alpha + rs;
         // P (single buffer) and O may be touched only once the previous P.V is done.
         if (g > 0) {
-          const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
+          const bool got_o = wait_bar<kDcColdReport>(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got_o)) {
             ok = false;
@@ -992,7 +1003,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
       // ---------------- epilogue of this piece
       l += __shfl_xor_sync(0xffffffffu, l, 16);
       if (sd.z > sd.y) {
-        const bool got_o = wait_bar(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
+        const bool got_o = wait_bar<kDcColdReport>(b_od, (g - 1) & 1, abort_flag, hdr, kDSiteODone, p.wait_ns);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got_o)) break;
         tc_fence_after();

@@ -403,6 +403,18 @@ bool decode_gqa_eligible(mxfa_dtype_t dt, int Hq, int Hkv, int Dqk, int Dv, int 
          (k_rs * 2) % 16 == 0 && (v_rs * 2) % 16 == 0;
 }
 
+// Multiplier and shift of div_u for the divisor d >= 1 (d < 1 is taken as 1).
+DivU make_divu(int d) {
+  d = std::max(d, 1);
+  int l = 0;
+  while ((1ll << l) < d) ++l;
+  DivU q;
+  q.sh = 31u + (uint32_t)l;
+  q.m = (uint32_t)(((1ull << q.sh) + (uint64_t)d - 1) / (uint64_t)d);
+  q.d = d;
+  return q;
+}
+
 // Split schedule in the workspace for `heads` = Hkv * subs decode sequences
 // (head groups) per batch entry.
 DecodeSched decode_sched(const AttnParams &p, int heads, int subs, int num_splits, int dv, int keys, void *ws,
@@ -412,6 +424,8 @@ DecodeSched decode_sched(const AttnParams &p, int heads, int subs, int num_split
   DecodeSched s;
   s.heads = heads;
   s.subs = subs;
+  s.by_hkv = make_divu(heads / std::max(subs, 1));
+  s.by_bh = make_divu(p.batch * (heads / std::max(subs, 1)));
   s.keys = keys;
   s.n_tiles = reinterpret_cast<int *>(base + w.n_tiles);
   s.tile_pre = reinterpret_cast<int *>(base + w.tile_pre);

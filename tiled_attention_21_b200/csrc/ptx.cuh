@@ -57,7 +57,9 @@ __device__ __forceinline__ bool mbar_wait_hint(uint32_t bar, uint32_t parity, ui
 // Bounded wait for the phase of parity `parity` of `bar` to complete.
 // Gives up when the CTA-wide abort flag is raised by another role, or when
 // `budget_ns` of %globaltimer run out (then records MXFA_ERR_TIMEOUT with
-// `site` and raises the abort flag).  Returns false when it gave up.
+// `site`, through report_error_cold when kColdReport, and raises the abort
+// flag).  Returns false when it gave up.
+template <bool kColdReport = false>
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag, WsHeader *hdr,
                                          uint32_t site, uint64_t budget_ns) {
   if (mbar_test(bar, parity)) return true;
@@ -66,7 +68,8 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     if (mbar_wait_hint(bar, parity, 1000000u)) return true;  // sleeps up to 1 ms
     if (*abort_flag) return false;
     if (global_ns() - t0 > budget_ns) {
-      report_error(hdr, kStatusTimeout, site);
+      if constexpr (kColdReport) report_error_cold(hdr, kStatusTimeout, site);
+      else report_error(hdr, kStatusTimeout, site);
       *abort_flag = 1;
       return false;
     }
