@@ -40,10 +40,11 @@
 //               row, then O_t's TMEM columns go back to the MMA issuer.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 after it.
 //
-// Every wait is bounded (see wait_bar); a wait that runs out records
-// MXFA_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag, and all
-// roles skip to the common teardown, which drains the TMA loads and MMAs
-// this CTA issued before TMEM is released.
+// Every wait is bounded (see wait_bar_flag); a wait that runs out leaves its
+// site in the CTA-wide abort flag, all roles skip to the common teardown,
+// which drains the TMA loads and MMAs this CTA issued before TMEM is
+// released, and thread 0 records MXFA_ERR_TIMEOUT with that site in the
+// workspace.
 #pragma once
 
 #include <type_traits>
@@ -209,23 +210,15 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// Largest (NEG: smallest) of N scores, keys >= lim excluded when MASKED
-// (an empty set gives -inf, NEG: +inf); four independent chains of
-// three-input maxima / minima.
-template <bool MASKED, bool NEG, int N>
-__device__ __forceinline__ float row_ext(const uint32_t (&sr)[N], int lim) {
-  constexpr float kEmpty = NEG ? INFINITY : -INFINITY;
-  float m4[4] = {kEmpty, kEmpty, kEmpty, kEmpty};
+// Largest of N scores (-inf for none: masked keys are set to -inf before);
+// four independent chains of three-input maxima.
+template <int N>
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[N]) {
+  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int q = 0; q < N; q += 2) {
-    float a = __uint_as_float(sr[q]), b = __uint_as_float(sr[q + 1]);
-    if (MASKED) {
-      a = q < lim ? a : kEmpty;
-      b = q + 1 < lim ? b : kEmpty;
-    }
-    m4[(q >> 1) & 3] = NEG ? fmin3(m4[(q >> 1) & 3], a, b) : fmax3(m4[(q >> 1) & 3], a, b);
-  }
-  return NEG ? fmin3(fminf(m4[0], m4[1]), m4[2], m4[3]) : fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+  for (int q = 0; q < N; q += 2)
+    m4[(q >> 1) & 3] = fmax3(m4[(q >> 1) & 3], __uint_as_float(sr[q]), __uint_as_float(sr[q + 1]));
+  return fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
 }
 
 // P = 2^(c*s - base) for N scores, written into TMEM at taddr as packed
@@ -364,7 +357,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       UnitInfo ui;
       for (int it = 0; ok && unit_at(p, it, cta, grid, n_units, ui); ++it) {
         const int nmax = max(ui.n[0], ui.n[1]);
-        if (it > 0 && !wait_bar(b_qe, (it - 1) & 1, abort_flag, hdr, kSiteQEmpty, p.wait_ns)) break;
+        if (it > 0 && !wait_bar_flag(b_qe, (it - 1) & 1, abort_flag, kSiteQEmpty, p.wait_ns)) break;
         mbar_arrive_expect_tx(b_qf, 2 * Cfg::kTileBytes);
         const int qrow = ui.sr.q0 + ui.m * kTcUnitRows;
 #pragma unroll
@@ -377,7 +370,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         for (int j = 0; j < nmax && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv, ++ring) {
             const int s = ring % Cfg::kSlots;
-            if (!wait_bar(b_se(s), ((ring / Cfg::kSlots) & 1) ^ 1, abort_flag, hdr, kSiteSlotEmpty, p.wait_ns)) {
+            if (!wait_bar_flag(b_se(s), ((ring / Cfg::kSlots) & 1) ^ 1, abort_flag, kSiteSlotEmpty, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -409,8 +402,8 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     // warp-uniformly; one elected lane issues each tcgen05 operation.
     const bool leader = elect_one();
     // every lane waits; the warp gives up together if any lane gave up
-    auto wait_warp = [&](uint32_t bar, uint32_t parity, volatile int *ab, WsHeader *h, uint32_t site) {
-      return __all_sync(0xffffffffu, wait_bar(bar, parity, ab, h, site, p.wait_ns));
+    auto wait_warp = [&](uint32_t bar, uint32_t parity, uint32_t site) {
+      return __all_sync(0xffffffffu, wait_bar_flag(bar, parity, abort_flag, site, p.wait_ns));
     };
     {
       constexpr uint32_t idesc_s = make_idesc_f16(BF16, kTcBlockM, kTcBlockN, false, false);
@@ -447,7 +440,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       UnitInfo ui;
       for (; ok && unit_at(p, it, cta, grid, n_units, ui); ++it) {
         const int nmax = max(ui.n[0], ui.n[1]);
-        if (!wait_warp(b_qf, it & 1, abort_flag, hdr, kSiteQFull)) break;
+        if (!wait_warp(b_qf, it & 1, kSiteQFull)) break;
         tc_fence_after();
         if (nmax == 0) {
           if (leader) mma_commit(b_qe);
@@ -456,7 +449,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         // prologue: S_t(0)
         {
           const int ks = ring % Cfg::kSlots;
-          if (!wait_warp(b_sf(ks), (ring / Cfg::kSlots) & 1, abort_flag, hdr, kSiteSlotFull)) break;
+          if (!wait_warp(b_sf(ks), (ring / Cfg::kSlots) & 1, kSiteSlotFull)) break;
           ++ring;
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
@@ -466,7 +459,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         }
         for (int j = 0; j < nmax && ok; ++j) {
           const int vs = ring % Cfg::kSlots;
-          if (!wait_warp(b_sf(vs), (ring / Cfg::kSlots) & 1, abort_flag, hdr, kSiteSlotFull)) {
+          if (!wait_warp(b_sf(vs), (ring / Cfg::kSlots) & 1, kSiteSlotFull)) {
             ok = false;
             break;
           }
@@ -483,13 +476,13 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
           }
           for (int t = 0; t < 2 && ok; ++t) {
             if (j >= ui.n[t]) continue;
-            if (!wait_warp(smem_u32(&ctrl->p_full[t]), p_cnt[t] & 1, abort_flag, hdr, kSitePFull)) {
+            if (!wait_warp(smem_u32(&ctrl->p_full[t]), p_cnt[t] & 1, kSitePFull)) {
               ok = false;
               break;
             }
             ++p_cnt[t];
             if (j == 0 && o_uses[t] > 0 &&
-                !wait_warp(smem_u32(&ctrl->o_empty[t]), (o_uses[t] - 1) & 1, abort_flag, hdr, kSiteOEmpty)) {
+                !wait_warp(smem_u32(&ctrl->o_empty[t]), (o_uses[t] - 1) & 1, kSiteOEmpty)) {
               ok = false;
               break;
             }
@@ -497,7 +490,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
             issue_pv(t, vs, j > 0, j + 1 == ui.n[t]);
             if (j + 1 < ui.n[t]) {
               if (!kwaited) {
-                if (!wait_warp(b_sf(ks), kph, abort_flag, hdr, kSiteSlotFull)) {
+                if (!wait_warp(b_sf(ks), kph, kSiteSlotFull)) {
                   ok = false;
                   break;
                 }
@@ -535,10 +528,12 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     const int bar_id = 1 + sub;     // the four warps of this sub-partition
     constexpr int OC = D / 4;       // output columns per thread
     const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16);
+    // A negative scale is handled by negating the scores in registers and
+    // using |scale*log2 e| (c*s = |c|*(-s)), so the row maximum has one form.
     const bool neg = p.scale_log2 < 0.f;
-    const float c = p.scale_log2;
+    const float c = fabsf(p.scale_log2);
     float *x_mine = &ctrl->xchg[g][r];
-    uint32_t s_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
+    uint32_t s_cnt[2] = {0, 0};
     int it = 0;
     bool ok = true;
     UnitInfo ui;
@@ -550,7 +545,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         // the exchange area holds the previous unit's row sums until the
         // epilogue warpgroup has taken them
         bool lf = true;
-        if (it > 0) lf = wait_bar(smem_u32(&ctrl->l_free), (it - 1) & 1, abort_flag, hdr, kSiteLFree, p.wait_ns);
+        if (it > 0) lf = wait_bar_flag(smem_u32(&ctrl->l_free), (it - 1) & 1, abort_flag, kSiteLFree, p.wait_ns);
         __syncwarp();
         if (bar_or(bar_id, 128, !__all_sync(0xffffffffu, lf))) break;
       }
@@ -566,7 +561,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
           // A failed wait does not leave the loop here: the four warps of the
           // sub-partition first agree on it at the next named barrier, so
           // none is left waiting there for a warp that has gone.
-          const bool got_s = wait_bar(smem_u32(&ctrl->s_full[t]), s_cnt[t] & 1, abort_flag, hdr, kSiteSFull, p.wait_ns);
+          const bool got_s = wait_bar_flag(smem_u32(&ctrl->s_full[t]), s_cnt[t] & 1, abort_flag, kSiteSFull, p.wait_ns);
           __syncwarp();
           const bool wok = __all_sync(0xffffffffu, got_s);
           ++s_cnt[t];
@@ -576,10 +571,19 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
           const bool masked = __any_sync(0xffffffffu, lim < 32);
           uint32_t sa[32];
           tmem_ld32(s_addr, sa);
-          // this group's largest c*s (a negative c turns the largest into the smallest s)
-          const float ext = neg ? (masked ? row_ext<true, true, 32>(sa, lim) : row_ext<false, true, 32>(sa, lim))
-                                : (masked ? row_ext<true, false, 32>(sa, lim) : row_ext<false, false, 32>(sa, lim));
-          const float pm = (ext == (neg ? INFINITY : -INFINITY)) ? -INFINITY : ext * c;
+          if (neg) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sa[e] ^= 0x80000000u;
+          }
+          if (masked) {  // keys >= lim to -inf (their P is set to 0 by exp_store as well)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sa[e] = e < lim ? sa[e] : 0xff800000u;
+          }
+          // this group's largest c*s.  One form of the reduction for all
+          // tiles: with variants for masked tiles and negative scales the
+          // softmax loop was longer and missed more in the instruction cache.
+          const float ext = row_max<32>(sa);
+          const float pm = (ext == -INFINITY) ? -INFINITY : ext * c;
           float alpha = 1.f;
           bool need = false;
           // Fast path: the stale base still bounds every group of every row
@@ -631,7 +635,6 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&ctrl->p_full[t]));
-          ++pv_cnt[t];
         }
       }
       if (!ok) break;
@@ -670,7 +673,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
     bool ok = true;
     UnitInfo ui;
     for (int it = 0; ok && unit_at(p, it, cta, grid, n_units, ui); ++it) {
-      const bool got_l = wait_bar(smem_u32(&ctrl->l_ready), it & 1, abort_flag, hdr, kSiteLReady, p.wait_ns);
+      const bool got_l = wait_bar_flag(smem_u32(&ctrl->l_ready), it & 1, abort_flag, kSiteLReady, p.wait_ns);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got_l)) break;
       const float lt0 = ctrl->xchg[0][r], lt1 = ctrl->xchg[1][r];
@@ -683,7 +686,7 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
         const bool valid = i < ui.sr.sq;
         T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(ui.sr.q0 + i) * p.o_rs + (int64_t)ui.h * p.o_hs;
         if (ui.n[t] > 0) {
-          const bool got_o = wait_bar(smem_u32(&ctrl->o_done[t]), o_cnt[t] & 1, abort_flag, hdr, kSiteODone, p.wait_ns);
+          const bool got_o = wait_bar_flag(smem_u32(&ctrl->o_done[t]), o_cnt[t] & 1, abort_flag, kSiteODone, p.wait_ns);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got_o)) {
             ok = false;
@@ -725,6 +728,8 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
 
   __syncwarp();  // the single-lane roles rejoin their warps before the CTA barrier
   __syncthreads();
+  // a wait that gave up left its site in the abort flag
+  if (threadIdx.x == 0 && ctrl->abort) report_error(hdr, kStatusTimeout, (uint32_t)ctrl->abort);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

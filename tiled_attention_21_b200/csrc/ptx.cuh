@@ -76,6 +76,27 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// The same wait for a kernel that reports once, in its teardown: a wait that
+// runs out records `site` in the CTA-wide abort flag (the first site wins;
+// any nonzero value makes the other roles give up) and touches no global
+// memory, so the give-up path that every wait site inlines is one
+// shared-memory atomic.  The prefill kernel uses it: its warps run with
+// setmaxnreg-lowered budgets, so its reports cannot be calls, and the inline
+// global report at each of its waits cost about 1 % of its time.
+__device__ __forceinline__ bool wait_bar_flag(uint32_t bar, uint32_t parity, volatile int *abort_flag, uint32_t site,
+                                              uint64_t budget_ns) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_wait_hint(bar, parity, 1000000u)) return true;  // sleeps up to 1 ms
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > budget_ns) {
+      atomicCAS(const_cast<int *>(abort_flag), 0, (int)site);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
