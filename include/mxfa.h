@@ -125,8 +125,7 @@ mxfa_status_t mxfa_attn_varlen_fwd(const void *q, const void *k, const void *v, 
  *     above 1 MiB, e.g. very large batch x max_seqlen_q) is rejected with
  *     MXFA_ERR_WORKSPACE and nothing is launched.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress) with that device current.
  *   - Calls share the one array: calls that overlap on the GPU (different
  *     streams without ordering, or several host threads) race and must not
  *     be issued; order them on one stream.
