@@ -99,6 +99,16 @@ def test_scale_zero_and_negative():
         check_full(p)
 
 
+def test_negative_scale_masked_tiles():
+    """A negative scale on the tensor-core path (the scores are negated in
+    registers and |scale| is used): causal diagonal tiles, a ragged last
+    tile, Sq != Sk, D = 64 and f16, and a varlen grouped-query batch."""
+    check_full(workloads.batched(15, 2, 300, 300, 4, 2, 64, "f16", True, scale=-0.11))
+    check_full(workloads.batched(15, 1, 200, 333, 4, 4, 128, "bf16", False, scale=-0.3))
+    check_full(workloads.batched(15, 1, 333, 200, 2, 1, 128, "bf16", True, scale=-0.05))
+    check_full(workloads.varlen(15, [129, 1, 300], [129, 7, 300], 8, 2, 128, "bf16", True, scale=-0.15))
+
+
 def test_large_scores_x50():
     """q, k scaled by 50 (oxillama-runtime flash_attention.rs,
     test_flash_attention_numerical_stability): O finite and within tolerance.
