@@ -102,11 +102,14 @@ def test_scale_zero_and_negative():
 def test_negative_scale_masked_tiles():
     """A negative scale on the tensor-core path (the scores are negated in
     registers and |scale| is used): causal diagonal tiles, a ragged last
-    tile, Sq != Sk, D = 64 and f16, and a varlen grouped-query batch."""
+    tile, Sq != Sk, D = 64 and f16, and a varlen grouped-query batch.  The
+    scales stay near head_dim^-0.5: at |scale| = 0.3 with D = 128 the
+    softmax is so peaked that the oracle rounded to bf16 is already 0.8-1.2e-2
+    from the oracle, beyond the 1e-2 bound for either sign."""
     check_full(workloads.batched(15, 2, 300, 300, 4, 2, 64, "f16", True, scale=-0.11))
-    check_full(workloads.batched(15, 1, 200, 333, 4, 4, 128, "bf16", False, scale=-0.3))
+    check_full(workloads.batched(15, 1, 200, 333, 4, 4, 128, "bf16", False, scale=-0.1))
     check_full(workloads.batched(15, 1, 333, 200, 2, 1, 128, "bf16", True, scale=-0.05))
-    check_full(workloads.varlen(15, [129, 1, 300], [129, 7, 300], 8, 2, 128, "bf16", True, scale=-0.15))
+    check_full(workloads.varlen(15, [129, 1, 300], [129, 7, 300], 8, 2, 128, "bf16", True, scale=-0.09))
 
 
 def test_large_scores_x50():
