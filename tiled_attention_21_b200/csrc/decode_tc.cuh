@@ -1080,6 +1080,7 @@ attn_decode_tc_kernel(const __grid_constant__ AttnParams p, const DecodeSched s,
 // not split (stored directly by the decode kernel) costs one load, and when
 // no sequence was split or left empty the kernel returns at once.
 constexpr int kDcCombineThreads = 256;
+constexpr int kDcCombineBatch = 4;  // pieces whose partials one thread loads in one round
 template <typename T, int DV>
 __global__ void __launch_bounds__(kDcCombineThreads) decode_combine_kernel(const AttnParams p, const DecodeSched s,
                                                                            int n_seq) {
@@ -1092,30 +1093,51 @@ __global__ void __launch_bounds__(kDcCombineThreads) decode_combine_kernel(const
   for (int64_t unit = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; unit < n_units;
        unit += (int64_t)gridDim.x * blockDim.x) {
     const int r = (int)(unit % R), c4 = (int)((unit / R) % C4), v = (int)(unit / ((int64_t)R * C4));
-    const int cnt = s.seg_cnt[v];
+    // The sequence's piece count, first piece and query range are loaded in
+    // one round, then (up to kDcCombineBatch pieces) every piece's (m, l) and
+    // accumulator in a second one: the kernel's time is its chain of
+    // dependent loads.  The sums run in piece order either way.
+    const DcSeq sq = dc_seq(p, s, v);
+    const int b = sq.b, gh = sq.gh;
+    const int cnt = s.seg_cnt[v], base = s.seg_base[v];
+    const int2 qr = dc_q(p, b);
     // not split: stored directly by the decode kernel (a sequence with no
     // piece, cnt = 0, is written here: O = 0, LSE = -inf)
     if (cnt == 1) continue;
-    const DcSeq sq = dc_seq(p, s, v);
-    const int b = sq.b, gh = sq.gh;
-    const int2 qr = dc_q(p, b);
     if (r >= qr.y * G) continue;
-    const int base = s.seg_base[v];
     float M = -INFINITY;
-    for (int i = 0; i < cnt; ++i) M = fmaxf(M, s.part_ml[(int64_t)(base + i) * kDcRows + r].x);
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
+    auto add = [&](float2 ml, float4 a) {
+      const float w = ex2(ml.x - M);  // 0 for a piece that saw no visible key
+      L += w * ml.y;
+      acc.x = fmaf(w, a.x, acc.x);
+      acc.y = fmaf(w, a.y, acc.y);
+      acc.z = fmaf(w, a.z, acc.z);
+      acc.w = fmaf(w, a.w, acc.w);
+    };
+    if (cnt <= kDcCombineBatch) {
+      float2 ml[kDcCombineBatch];
+      float4 a[kDcCombineBatch];
+#pragma unroll
+      for (int i = 0; i < kDcCombineBatch; ++i)
+        if (i < cnt) {
+          ml[i] = s.part_ml[(int64_t)(base + i) * kDcRows + r];
+          a[i] = *dc_pacc<DV>(s, base + i, r, c4);
+        }
+#pragma unroll
+      for (int i = 0; i < kDcCombineBatch; ++i)
+        if (i < cnt) M = fmaxf(M, ml[i].x);
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int i = 0; i < kDcCombineBatch; ++i)
+          if (i < cnt) add(ml[i], a[i]);
+      }
+    } else {
+      for (int i = 0; i < cnt; ++i) M = fmaxf(M, s.part_ml[(int64_t)(base + i) * kDcRows + r].x);
+      if (M != -INFINITY) {
 #pragma unroll 4
-      for (int i = 0; i < cnt; ++i) {
-        const float2 ml = s.part_ml[(int64_t)(base + i) * kDcRows + r];
-        const float w = ex2(ml.x - M);  // 0 for a piece that saw no visible key
-        L += w * ml.y;
-        const float4 a = *dc_pacc<DV>(s, base + i, r, c4);
-        acc.x = fmaf(w, a.x, acc.x);
-        acc.y = fmaf(w, a.y, acc.y);
-        acc.z = fmaf(w, a.z, acc.z);
-        acc.w = fmaf(w, a.w, acc.w);
+        for (int i = 0; i < cnt; ++i) add(s.part_ml[(int64_t)(base + i) * kDcRows + r], *dc_pacc<DV>(s, base + i, r, c4));
       }
     }
     const int tok = qr.x + r / G, h = gh * G + r % G;
