@@ -284,8 +284,10 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
       n = (len + s.keys - 1) / s.keys;
       if (dc_q(p, e).y <= 0) n = 0;  // no queries: nothing to compute
       s.n_tiles[b] = n;
-      atomicMax(&max_n, n);
     }
+    // one shared atomic per warp (all lanes reach here; n = 0 past B)
+    const int wmax = __reduce_max_sync(0xffffffffu, n);
+    if ((tid & 31) == 0 && wmax > 0) atomicMax(&max_n, wmax);
     int incl, total;
     Scan(tmp).InclusiveSum(n, incl, total);
     if (b < B) s.tile_pre[b + 1] = carry + incl;
@@ -345,7 +347,8 @@ __global__ void __launch_bounds__(1024) decode_prep_kernel(const AttnParams p, D
     const int b = base + tid;
     const int k = b < B ? pieces(b) : 0;
     if (b < B) s.seg_cnt[b] = k;
-    if (b < B && k != 1) atomicAdd(&n_multi, 1);
+    const int wmulti = (int)__reduce_add_sync(0xffffffffu, (b < B && k != 1) ? 1u : 0u);
+    if ((tid & 31) == 0 && wmulti > 0) atomicAdd(&n_multi, wmulti);
     int incl, total;
     Scan(tmp).InclusiveSum(k, incl, total);
     if (b < B) s.seg_base[b] = carry + incl - k;
