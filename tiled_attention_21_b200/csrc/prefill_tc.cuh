@@ -616,19 +616,15 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
             // Rescale O_t.  PV_t(j-1), its latest accumulation, is complete:
             // it was issued before S_t(j), and the commit that signalled
             // S_t(j) tracks every earlier MMA of the issuing thread.
+            // (rare: 16-column pieces in a rolled loop, for code size)
             const uint32_t oa = trow + 2 * kTcBlockN + t * D + g * OC;
-            if constexpr (OC == 32) {
-              uint32_t ov[32];
-              tmem_ld32(oa, ov);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-              tmem_st32(oa, ov);
-            } else {
+#pragma unroll 1
+            for (int h16 = 0; h16 < OC / 16; ++h16) {
               uint32_t ov[16];
-              tmem_ld16(oa, ov);
+              tmem_ld16(oa + h16 * 16, ov);
 #pragma unroll
               for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-              tmem_st16(oa, ov);
+              tmem_st16(oa + h16 * 16, ov);
             }
             tmem_wait_st();
           }
@@ -679,23 +675,29 @@ attn_fwd_tc_kernel(const __grid_constant__ AttnParams p, const __grid_constant__
       const float lt0 = ctrl->xchg[0][r], lt1 = ctrl->xchg[1][r];
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&ctrl->l_free));
-#pragma unroll
+      // Rolled loops (the tile state selected, not indexed): this warpgroup
+      // shares the SM sub-partitions with the softmax warps, and its code,
+      // run once per unit, is kept small so the softmax loop stays in the
+      // instruction cache (unrolled over both tiles and all column chunks it
+      // cost 1.5-2 % on the 2K and varlen workloads).
+#pragma unroll 1
       for (int t = 0; t < 2; ++t) {
         const float lt = t ? lt1 : lt0;
         const int i = ui.m * kTcUnitRows + t * kTcBlockM + r;
         const bool valid = i < ui.sr.sq;
         T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(ui.sr.q0 + i) * p.o_rs + (int64_t)ui.h * p.o_hs;
-        if (ui.n[t] > 0) {
-          const bool got_o = wait_bar_flag(smem_u32(&ctrl->o_done[t]), o_cnt[t] & 1, abort_flag, kSiteODone, p.wait_ns);
+        if ((t ? ui.n[1] : ui.n[0]) > 0) {
+          const uint32_t oc = t ? o_cnt[1] : o_cnt[0];
+          const bool got_o = wait_bar_flag(smem_u32(&ctrl->o_done[t]), oc & 1, abort_flag, kSiteODone, p.wait_ns);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got_o)) {
             ok = false;
             break;
           }
-          ++o_cnt[t];
+          if (t) o_cnt[1] = oc + 1; else o_cnt[0] = oc + 1;
           tc_fence_after();
           const float inv = lt > 0.f ? 1.f / lt : 0.f;
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < D / 16; ++c) {
             uint32_t ov[16], pk[8];
             tmem_ld16(trow + 2 * kTcBlockN + t * D + c * 16, ov);
