@@ -248,24 +248,33 @@ std::atomic<int> g_keep_merge_counters{0};
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- launchers
-template <typename T, int DVL>
-mxfa_status_t launch_simt_dv(const AttnParams &p, dim3 grid, size_t smem, cudaStream_t st) {
-  auto k = attn_fwd_simt_kernel<T, DVL>;
+template <typename T, int DVL, int KS>
+mxfa_status_t launch_simt_dv(const AttnParams &p, dim3 grid, cudaStream_t st) {
+  auto k = attn_fwd_simt_kernel<T, DVL, KS>;
+  const size_t smem = simt_smem_bytes(p.dqk, p.dv, KS);
   MXFA_TRY(ensure_smem(reinterpret_cast<const void *>(k), smem));
-  k<<<grid, kSimtWarps * 32, smem, st>>>(p);
+  k<<<grid, kSimtWarps * 32 * KS, smem, st>>>(p);
   MXFA_CUDA(cudaGetLastError());
   return MXFA_OK;
 }
 
+// Four key splits per block when the blocks cover at most half the SMs and
+// the keys span more than one tile: a row's tiles are then worked on side by
+// side instead of one after another (head dims up to 128, where four staged
+// tiles fit in shared memory and 1024 threads in the registers).
 template <typename T>
 mxfa_status_t launch_simt(const AttnParams &p, int max_rows_per_seq_head, cudaStream_t st) {
-  const size_t smem = simt_smem_bytes(p.dqk, p.dv);
   const int G = p.hq / p.hkv;
   dim3 grid((unsigned)((max_rows_per_seq_head * (int64_t)G + kSimtWarps - 1) / kSimtWarps), p.hkv, p.batch);
   if (grid.x == 0) return MXFA_OK;
-  if (p.dv <= 64) return launch_simt_dv<T, 2>(p, grid, smem, st);
-  if (p.dv <= 128) return launch_simt_dv<T, 4>(p, grid, smem, st);
-  return launch_simt_dv<T, 16>(p, grid, smem, st);
+  int sms = 0;
+  MXFA_TRY(sm_count(&sms));
+  const int64_t blocks = (int64_t)grid.x * grid.y * grid.z;
+  if (2 * blocks <= sms && p.max_sk > kSimtKeys && p.dqk <= 128 && p.dv <= 128)
+    return p.dv <= 64 ? launch_simt_dv<T, 2, 4>(p, grid, st) : launch_simt_dv<T, 4, 4>(p, grid, st);
+  if (p.dv <= 64) return launch_simt_dv<T, 2, 1>(p, grid, st);
+  if (p.dv <= 128) return launch_simt_dv<T, 4, 1>(p, grid, st);
+  return launch_simt_dv<T, 16, 1>(p, grid, st);
 }
 
 mxfa_status_t launch_simt_any(mxfa_dtype_t dt, const AttnParams &p, int max_rows, cudaStream_t st) {

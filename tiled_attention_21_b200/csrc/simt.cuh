@@ -21,29 +21,39 @@
 
 namespace mxfa {
 
-constexpr int kSimtWarps = 8;
+constexpr int kSimtWarps = 8;   // rows per block
 constexpr int kSimtKeys = 32;
-constexpr int kSimtStage = 8;  // loads in flight per thread while a tile is staged
 
+// Key splits per block: KS = 1, or 4 for problems with few blocks (the KS
+// warps of a row take interleaved 32-key tiles and merge their partial
+// (max, sum, accumulator) at the end, so a short sequence is one tile deep
+// instead of four).  Loads in flight per thread while tiles are staged.
+template <int KS>
+constexpr int simt_stage() { return KS == 1 ? 8 : 4; }
 
-__host__ __device__ inline size_t simt_smem_bytes(int dqk, int dv) {
-  return sizeof(float) * ((size_t)kSimtWarps * dqk + (size_t)kSimtKeys * (dqk + 1) + (size_t)kSimtKeys * dv);
+__host__ __device__ inline size_t simt_smem_bytes(int dqk, int dv, int ks = 1) {
+  const size_t tiles = (size_t)ks * ((size_t)kSimtKeys * (dqk + 1) + (size_t)kSimtKeys * dv);
+  const size_t merge = ks > 1 ? (size_t)(ks - 1) * kSimtWarps * (dv + 2) : 0;  // reuses the tile area
+  return sizeof(float) * ((size_t)kSimtWarps * dqk + (tiles > merge ? tiles : merge));
 }
 
-template <typename T, int DV_PER_LANE>
-__global__ void __launch_bounds__(kSimtWarps * 32, 2)
+template <typename T, int DV_PER_LANE, int KS>
+__global__ void __launch_bounds__(kSimtWarps * 32 * KS, KS == 1 ? 2 : 1)
 attn_fwd_simt_kernel(const AttnParams p) {
   extern __shared__ float smem[];
   const int dqk = p.dqk, dv = p.dv;
+  const int tile_floats = kSimtKeys * (dqk + 1) + kSimtKeys * dv;
   float *qs = smem;                                   // [kSimtWarps][dqk]
-  float *ks = qs + kSimtWarps * dqk;                  // [kSimtKeys][dqk + 1]
-  float *vs = ks + kSimtKeys * (dqk + 1);             // [kSimtKeys][dv]
+  float *tiles = qs + kSimtWarps * dqk;               // KS x ([kSimtKeys][dqk + 1], [kSimtKeys][dv])
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rw = warp % kSimtWarps, sp = warp / kSimtWarps;  // row slot, key split
+  float *ks = tiles + sp * tile_floats;               // this split's K tile
+  float *vs = ks + kSimtKeys * (dqk + 1);             // and V tile
   const int b = blockIdx.z, g = blockIdx.y;
   const SeqRange sr = seq_range(p, b);
   const int G = p.hq / p.hkv;
-  const int row = blockIdx.x * kSimtWarps + warp;    // flattened (query, head-in-group)
+  const int row = blockIdx.x * kSimtWarps + rw;       // flattened (query, head-in-group)
   const int n_rows = sr.sq * G;
   if (blockIdx.x * kSimtWarps >= n_rows) return;     // whole block idle (uniform)
 
@@ -57,7 +67,8 @@ attn_fwd_simt_kernel(const AttnParams p) {
   const int block_keys = visible_keys(last_row / G, sr.sq, sr.sk, p.causal);
 
   const T *qrow = reinterpret_cast<const T *>(p.q) + (int64_t)(sr.q0 + i) * p.q_rs + (int64_t)h * p.q_hs;
-  for (int d = lane; d < dqk; d += 32) qs[warp * dqk + d] = active ? to_f32(qrow[d]) : 0.f;
+  if (sp == 0)
+    for (int d = lane; d < dqk; d += 32) qs[rw * dqk + d] = active ? to_f32(qrow[d]) : 0.f;
 
   float m = -INFINITY, l = 0.f;
   float acc[DV_PER_LANE], acc2[DV_PER_LANE];
@@ -68,70 +79,88 @@ attn_fwd_simt_kernel(const AttnParams p) {
   const T *vbase = reinterpret_cast<const T *>(p.v) + (int64_t)g * p.v_hs;
 
   // K and V tiles are staged in 16-byte pieces: a thread issues a batch of
-  // independent loads before it converts and stores any of them, so a tile
-  // costs about one memory latency.  Rows are 16-byte aligned (the entry
-  // points check the pointers and strides), and dqk, dv are multiples of the
-  // eight or four elements of a piece.
+  // independent loads before it converts and stores any of them, so a group
+  // of KS tiles costs about one memory latency.  Rows are 16-byte aligned
+  // (the entry points check the pointers and strides), and dqk, dv are
+  // multiples of the eight or four elements of a piece.
   constexpr int kVec = 16 / sizeof(T);
-  constexpr int kBatch = kSimtStage * kSimtWarps * 32;
+  constexpr int kStage = simt_stage<KS>();
+  constexpr int kBatch = kStage * kSimtWarps * 32 * KS;
   const int kq = dqk / kVec, vq = dv / kVec;
-  const int n_pieces = kSimtKeys * (kq + vq);
-  // c / kq and c / vq as a multiply-high by ceil(2^32 / divisor): exact for
-  // c * divisor^2 < 2^32 (here c < 32 * 288 and divisors <= 144)
+  const int n_pieces = kSimtKeys * (kq + vq);          // per tile
+  // c / kq, c / vq and c / n_pieces as a multiply-high by ceil(2^32 / divisor):
+  // exact for c * divisor^2 < 2^32 (here c < KS * n_pieces <= 4 * 32 * 288
+  // and divisors <= 144 when KS = 1; c < 4 * 2048, divisors <= 2048 when KS = 4)
   const uint32_t mk = (uint32_t)(((1ull << 32) + kq - 1) / kq), mv = (uint32_t)(((1ull << 32) + vq - 1) / vq);
-  auto load = [&](int t, int base, uint4 (&w)[kSimtStage]) {
-    const int nk = min(kSimtKeys, block_keys - t);
+  const uint32_t mp = (uint32_t)(((1ull << 32) + n_pieces - 1) / n_pieces);
+  // piece c of the group: tile s = c / n_pieces, then a K or V row piece
+  auto locate = [&](int c, int &s, int &j, int &dc, bool &is_k) {
+    s = KS == 1 ? 0 : (int)__umulhi((uint32_t)c, mp);
+    const int cl = c - s * n_pieces;
+    is_k = cl < kSimtKeys * kq;
+    const int cv = is_k ? cl : cl - kSimtKeys * kq;
+    j = (int)__umulhi((uint32_t)cv, is_k ? mk : mv);
+    dc = cv - j * (is_k ? kq : vq);
+  };
+  auto load = [&](int t0, int base, uint4 (&w)[kStage]) {
 #pragma unroll
-    for (int u = 0; u < kSimtStage; ++u) {
-      const int c = base + u * kSimtWarps * 32;
+    for (int u = 0; u < kStage; ++u) {
+      const int c = base + u * kSimtWarps * 32 * KS;
       w[u] = make_uint4(0, 0, 0, 0);
-      if (c < kSimtKeys * kq) {
-        const int j = (int)__umulhi((uint32_t)c, mk), dc = c - j * kq;
-        if (j < nk) w[u] = *reinterpret_cast<const uint4 *>(kbase + (int64_t)(sr.k0 + t + j) * p.k_rs + dc * kVec);
-      } else if (c < n_pieces) {
-        const int cv = c - kSimtKeys * kq, j = (int)__umulhi((uint32_t)cv, mv), dc = cv - j * vq;
-        if (j < nk) w[u] = *reinterpret_cast<const uint4 *>(vbase + (int64_t)(sr.k0 + t + j) * p.v_rs + dc * kVec);
+      if (c < KS * n_pieces) {
+        int s, j, dc;
+        bool is_k;
+        locate(c, s, j, dc, is_k);
+        const int key = t0 + s * kSimtKeys + j;
+        if (key < block_keys && j < kSimtKeys)
+          w[u] = is_k ? *reinterpret_cast<const uint4 *>(kbase + (int64_t)(sr.k0 + key) * p.k_rs + dc * kVec)
+                      : *reinterpret_cast<const uint4 *>(vbase + (int64_t)(sr.k0 + key) * p.v_rs + dc * kVec);
       }
     }
   };
-  auto store = [&](int base, const uint4 (&w)[kSimtStage]) {
+  auto store = [&](int base, const uint4 (&w)[kStage]) {
 #pragma unroll
-    for (int u = 0; u < kSimtStage; ++u) {
-      const int c = base + u * kSimtWarps * 32;
-      const T *e = reinterpret_cast<const T *>(&w[u]);
-      if (c < kSimtKeys * kq) {
-        const int j = (int)__umulhi((uint32_t)c, mk), dc = c - j * kq;
+    for (int u = 0; u < kStage; ++u) {
+      const int c = base + u * kSimtWarps * 32 * KS;
+      if (c < KS * n_pieces) {
+        int s, j, dc;
+        bool is_k;
+        locate(c, s, j, dc, is_k);
+        float *kt = tiles + s * tile_floats, *vt = kt + kSimtKeys * (dqk + 1);
+        const T *e = reinterpret_cast<const T *>(&w[u]);
+        if (is_k) {
 #pragma unroll
-        for (int i = 0; i < kVec; ++i) ks[j * (dqk + 1) + dc * kVec + i] = to_f32(e[i]);
-      } else if (c < n_pieces) {
-        const int cv = c - kSimtKeys * kq, j = (int)__umulhi((uint32_t)cv, mv), dc = cv - j * vq;
+          for (int x = 0; x < kVec; ++x) kt[j * (dqk + 1) + dc * kVec + x] = to_f32(e[x]);
+        } else {
 #pragma unroll
-        for (int i = 0; i < kVec; ++i) vs[j * dv + dc * kVec + i] = to_f32(e[i]);
+          for (int x = 0; x < kVec; ++x) vt[j * dv + dc * kVec + x] = to_f32(e[x]);
+        }
       }
     }
   };
-  for (int t0 = 0; t0 < block_keys; t0 += kSimtKeys) {
-    __syncthreads();  // previous tile fully consumed (also orders the qs writes)
-    const int nk = min(kSimtKeys, block_keys - t0);
-    for (int base = threadIdx.x; base < n_pieces; base += kBatch) {
-      uint4 w[kSimtStage];
-      load(t0, base, w);
+  for (int tg = 0; tg < block_keys; tg += KS * kSimtKeys) {
+    __syncthreads();  // previous tiles fully consumed (also orders the qs writes)
+    for (int base = threadIdx.x; base < KS * n_pieces; base += kBatch) {
+      uint4 w[kStage];
+      load(tg, base, w);
       store(base, w);
     }
     __syncthreads();
+    const int t0 = tg + sp * kSimtKeys;  // this split's tile
     if (!active || t0 >= n_vis) continue;
+    const int nk = min(kSimtKeys, block_keys - t0);
 
     // score of key t0 + lane, in the log2 domain: four partial sums over
     // d mod 4 (dqk is a multiple of 4), so the FMA chain is a quarter as long
     const float *kr = ks + lane * (dqk + 1);
-    const float *qr = qs + warp * dqk;
+    const float *qr = qs + rw * dqk;
     float s4[4] = {0.f, 0.f, 0.f, 0.f};
     for (int d = 0; d < dqk; d += 4) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) s4[u] = fmaf(qr[d + u], kr[d + u], s4[u]);
     }
-    const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-    float x = (t0 + lane < n_vis) ? s * p.scale_log2 : -INFINITY;
+    const float sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+    float x = (t0 + lane < n_vis) ? sc * p.scale_log2 : -INFINITY;
 
     float tmax = x;
 #pragma unroll
@@ -164,6 +193,49 @@ attn_fwd_simt_kernel(const AttnParams p) {
       }
     }
   }
+#pragma unroll
+  for (int e = 0; e < DV_PER_LANE; ++e) acc[e] += acc2[e];
+
+  if constexpr (KS > 1) {
+    // Splits 1..KS-1 hand (m, l, acc) to split 0 through the tile area:
+    // O = sum_s acc_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), M = max_s m_s.
+    float *mg = tiles;  // [KS-1][kSimtWarps][dv + 2]
+    __syncthreads();    // every split is done with the tiles
+    if (active && sp > 0) {
+      float *slot = mg + ((sp - 1) * kSimtWarps + rw) * (dv + 2);
+      if (lane == 0) {
+        slot[dv] = m;
+        slot[dv + 1] = l;
+      }
+#pragma unroll
+      for (int e = 0; e < DV_PER_LANE; ++e) {
+        const int d = lane + 32 * e;
+        if (d < dv) slot[d] = acc[e];
+      }
+    }
+    __syncthreads();
+    if (!active || sp > 0) return;
+    float M = m;
+#pragma unroll
+    for (int q = 1; q < KS; ++q) M = fmaxf(M, mg[((q - 1) * kSimtWarps + rw) * (dv + 2) + dv]);
+    const float wm = (m == -INFINITY) ? 0.f : exp2f(m - M);  // a split that saw no key weighs 0
+    l *= wm;
+#pragma unroll
+    for (int e = 0; e < DV_PER_LANE; ++e) acc[e] *= wm;
+#pragma unroll
+    for (int q = 1; q < KS; ++q) {
+      const float *slot = mg + ((q - 1) * kSimtWarps + rw) * (dv + 2);
+      const float mq = slot[dv];
+      const float w = (mq == -INFINITY) ? 0.f : exp2f(mq - M);
+      l = fmaf(slot[dv + 1], w, l);
+#pragma unroll
+      for (int e = 0; e < DV_PER_LANE; ++e) {
+        const int d = lane + 32 * e;
+        if (d < dv) acc[e] = fmaf(slot[d], w, acc[e]);
+      }
+    }
+    m = M;
+  }
   if (!active) return;
 
   T *orow = reinterpret_cast<T *>(p.o) + (int64_t)(sr.q0 + i) * p.o_rs + (int64_t)h * p.o_hs;
@@ -171,7 +243,7 @@ attn_fwd_simt_kernel(const AttnParams p) {
 #pragma unroll
   for (int e = 0; e < DV_PER_LANE; ++e) {
     const int d = lane + 32 * e;
-    if (d < dv) orow[d] = from_f32<T>((acc[e] + acc2[e]) * inv);
+    if (d < dv) orow[d] = from_f32<T>(acc[e] * inv);
   }
   if (p.lse && lane == 0) {
     const float lse = l > 0.f ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
